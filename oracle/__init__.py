@@ -1,0 +1,41 @@
+"""CPU oracle for the flow-matching action-expert denoise loop.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import or call this
+package: only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` use it.  It shares no code with the
+CUDA library; the only module both sides use is ``synth`` (seeded inputs).
+
+Everything is plain numpy in float64 on the bf16-rounded inputs.  A library
+matmul serves as the dot-product step; there is no blocking, fusion or
+reordering beyond the definitions below.
+
+Functions and what pins them (tests under ``tests/test_oracle_*.py``):
+
+=====================  =========================================================
+``euler_integrate``    closed form of Euler on a linear field v = A x + b,
+                       exact-ODE error bound, A = 0 and N = 1 special cases
+``timestep_embedding`` t = 0 gives [1..1, 0..0]; first frequency is 1000 t;
+                       last frequency matches the base-10000 geometric series
+``rms_norm``           unit RMS at eps = 0, scale invariance, torch's rms_norm
+``modulate``           shift = scale = 0 is the identity
+``rope_half``          per-pair norm, position 0 identity, relative-position
+                       property, complex-multiplication form
+``gqa_attention``      torch SDPA (enable_gqa) in float64, brute-force score
+                       matrix, P = 0, constant-V rows, MHA case
+``linear``/``swiglu``  torch float64 linear / silu, SiLU(0) = 0
+``e4m3_*``             exhaustive code table, RNE ties, saturation, torch cast
+``dit_layer``          zero gates give the identity, joint prefix permutation
+                       invariance
+``velocity``/``denoise``  parity unpinned beyond the parts above: batch
+                       independence (bitwise), determinism
+=====================  =========================================================
+"""
+
+from .model import (  # noqa: F401
+    bf16_to_f64, t_schedule, timestep_embedding, silu, rms_norm, modulate, rope_half,
+    rope_positions_angles, gqa_attention, linear, swiglu, euler_integrate,
+    adaln_table, dit_layer, velocity, denoise, denoise_batch, OracleWeights,
+)
+from .fp8 import (  # noqa: F401
+    e4m3_decode, e4m3_encode, quantize_rowwise_e4m3, dequantize_rowwise_e4m3,
+)

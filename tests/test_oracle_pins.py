@@ -1,0 +1,427 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (no GPU).
+
+Each test ties an oracle function to something other than itself: a closed form, an
+invariant, a library routine computing the same textbook operation, brute force on tiny
+inputs, or a golden table written from a format definition.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle import fp8 as ofp8
+from synth import config, generate_weights, generate_inputs, f32_to_bf16_bits, bf16_bits_to_f32
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(1234)
+
+
+# ----------------------------------------------------------------- Euler sampler
+
+def _linear_field(n=7, seed=0):
+    rng = np.random.default_rng(seed)
+    a = rng.standard_normal((n, n))
+    a = a / np.linalg.norm(a, 2)            # spectral norm 1
+    b = rng.standard_normal(n)
+    x0 = rng.standard_normal(n)
+    return a, b, x0
+
+
+@pytest.mark.parametrize("n_steps", [1, 2, 4, 10, 37])
+def test_euler_linear_field_closed_form(n_steps):
+    a, b, x0 = _linear_field()
+    got = oracle.euler_integrate(x0, n_steps, lambda x, t: a @ x + b)
+    dt = -1.0 / n_steps
+    m = np.eye(7) + dt * a
+    want = np.linalg.matrix_power(m, n_steps) @ x0
+    for j in range(n_steps):
+        want = want + np.linalg.matrix_power(m, j) @ (dt * b)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_euler_converges_to_exact_flow_first_order():
+    a, b, x0 = _linear_field(seed=3)
+    ea = scipy.linalg.expm(-a)
+    exact = ea @ x0 + np.linalg.solve(a, (ea - np.eye(7)) @ b)
+    errs = []
+    for n in (64, 128, 256, 512):
+        got = oracle.euler_integrate(x0, n, lambda x, t: a @ x + b)
+        errs.append(np.max(np.abs(got - exact)))
+    ratios = [errs[i] / errs[i + 1] for i in range(3)]
+    for r in ratios:
+        assert 1.8 < r < 2.2, (errs, ratios)           # global error O(|dt|)
+    # the Euler bound |err| <= |dt| * C with C of order ||A|| e^{||A||} (||b|| + ||x||)
+    assert errs[0] < 64 ** -1 * 50
+
+
+def test_euler_zero_field_and_single_step():
+    _, b, x0 = _linear_field(seed=5)
+    got = oracle.euler_integrate(x0, 8, lambda x, t: b)
+    np.testing.assert_allclose(got, x0 - b, rtol=0, atol=1e-14)
+    seen = []
+
+    def v(x, t):
+        seen.append(t)
+        return np.sin(x) + t
+
+    got1 = oracle.euler_integrate(x0, 1, v)
+    assert seen == [1.0]
+    assert np.array_equal(got1, x0 - (np.sin(x0) + 1.0))
+
+
+def test_euler_time_grid_golden():
+    with open(os.path.join(GOLDEN, "euler_schedule.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for r in rows:
+        n, dt, ts = int(r[0]), float(r[1]), [float(x) for x in r[2:]]
+        got_ts, got_dt = oracle.t_schedule(n)
+        assert got_dt == dt
+        np.testing.assert_allclose(got_ts, ts, rtol=0, atol=1e-15)
+        seen = []
+        oracle.euler_integrate(np.zeros(1), n, lambda x, t: seen.append(t) or np.zeros(1))
+        np.testing.assert_allclose(seen, ts, rtol=0, atol=1e-15)
+
+
+# ----------------------------------------------------------------- time embedding
+
+def test_timestep_embedding_t0_and_identity():
+    e = oracle.timestep_embedding(0.0, 256)
+    assert np.array_equal(e, np.concatenate([np.ones(128), np.zeros(128)]))
+    for t in (1.0, 0.75, 0.1, 0.333):
+        e = oracle.timestep_embedding(t, 256)
+        # cos^2 + sin^2 = 1 pairs element i of each half at the same frequency
+        np.testing.assert_allclose(e[:128] ** 2 + e[128:] ** 2, 1.0, atol=1e-14)
+        # first frequency is 1: a_0 = 1000 t
+        assert math.isclose(e[0], math.cos(1000.0 * t), abs_tol=1e-12)
+        assert math.isclose(e[128], math.sin(1000.0 * t), abs_tol=1e-12)
+    # frequencies form a geometric series from 1 down to 10000^(-127/128)
+    t = 1e-4
+    e = oracle.timestep_embedding(t, 256)
+    ang = np.arctan2(e[128:], e[:128]) / (1000.0 * t)
+    ratio = ang[1:] / ang[:-1]
+    np.testing.assert_allclose(ratio, 10000.0 ** (-1.0 / 128), rtol=1e-9)
+
+
+def test_silu_values():
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    z = RNG.standard_normal(100) * 4
+    np.testing.assert_allclose(oracle.silu(z), F.silu(torch.tensor(z)).numpy(), rtol=1e-14, atol=1e-15)
+
+
+# ----------------------------------------------------------------- RMSNorm / modulate
+
+def test_rms_norm_unit_rms_and_scale_invariance():
+    h = RNG.standard_normal((5, 96)) * 3.0
+    y = oracle.rms_norm(h, eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(y * y, axis=1)), 1.0, atol=1e-12)
+    np.testing.assert_allclose(oracle.rms_norm(7.5 * h, eps=0.0), y, rtol=1e-12, atol=1e-13)
+    # textbook routine: torch's rms_norm with the same eps and no affine weight
+    want = F.rms_norm(torch.tensor(h), (96,), eps=1e-6).numpy()
+    np.testing.assert_allclose(oracle.rms_norm(h, 1e-6), want, rtol=1e-12, atol=1e-13)
+
+
+def test_modulate_identity_and_form():
+    u = RNG.standard_normal((3, 8))
+    z = np.zeros(8)
+    assert np.array_equal(oracle.modulate(u, z, z), u)
+    np.testing.assert_allclose(oracle.modulate(u, z, -np.ones(8)), 0.0)      # (1 + scale) form
+    s = RNG.standard_normal(8)
+    np.testing.assert_allclose(oracle.modulate(u, s, z), u + s)
+
+
+# ----------------------------------------------------------------- RoPE
+
+@pytest.mark.parametrize("hd", [8, 64, 256])
+def test_rope_invariants(hd):
+    x = RNG.standard_normal((6, 3, hd))
+    pos = np.arange(6) + 11.0
+    y = oracle.rope_half(x, pos)
+    half = hd // 2
+    np.testing.assert_allclose(x[..., :half] ** 2 + x[..., half:] ** 2,
+                               y[..., :half] ** 2 + y[..., half:] ** 2, rtol=1e-12)
+    np.testing.assert_allclose(oracle.rope_half(x, np.zeros(6)), x, rtol=0, atol=0)
+    # complex form: z_i = x_i + i x_{i+hd/2} rotated by e^{i theta}, theta = p * 10000^(-2i/hd)
+    z = x[..., :half] + 1j * x[..., half:]
+    th = pos[:, None, None] * 10000.0 ** (-2.0 * np.arange(half) / hd)[None, None, :]
+    zr = z * np.exp(1j * th)
+    np.testing.assert_allclose(y[..., :half], zr.real, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y[..., half:], zr.imag, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_relative_position():
+    hd = 32
+    q = RNG.standard_normal((1, 1, hd))
+    k = RNG.standard_normal((1, 1, hd))
+    for m, n, s in ((3, 7, 5), (0, 10, 100), (40, 2, 17)):
+        a = np.sum(oracle.rope_half(q, np.array([m * 1.0])) * oracle.rope_half(k, np.array([n * 1.0])))
+        b = np.sum(oracle.rope_half(q, np.array([m + s * 1.0])) * oracle.rope_half(k, np.array([n + s * 1.0])))
+        assert math.isclose(a, b, rel_tol=1e-10, abs_tol=1e-12)
+
+
+# ----------------------------------------------------------------- attention
+
+def _brute_attention(q, k, v):
+    """Score matrix written out element by element, kv heads materialised by repetition."""
+    T, nq, hd = q.shape
+    nkv = k.shape[1]
+    k_rep = np.repeat(k, nq // nkv, axis=1)
+    v_rep = np.repeat(v, nq // nkv, axis=1)
+    out = np.zeros_like(q)
+    for h in range(nq):
+        for i in range(T):
+            s = [sum(q[i, h, d] * k_rep[j, h, d] for d in range(hd)) / math.sqrt(hd)
+                 for j in range(k.shape[0])]
+            mx = max(s)
+            e = [math.exp(x - mx) for x in s]
+            z = sum(e)
+            for d in range(hd):
+                out[i, h, d] = sum(e[j] * v_rep[j, h, d] for j in range(k.shape[0])) / z
+    return out
+
+
+@pytest.mark.parametrize("nq,nkv", [(4, 2), (4, 1), (4, 4)])
+def test_attention_brute_force_and_sdpa(nq, nkv):
+    Ts, P, hd = 3, 5, 8
+    q = RNG.standard_normal((Ts, nq, hd))
+    k = RNG.standard_normal((P + Ts, nkv, hd))
+    v = RNG.standard_normal((P + Ts, nkv, hd))
+    got = oracle.gqa_attention(q, k, v)
+    np.testing.assert_allclose(got, _brute_attention(q, k, v), rtol=1e-12, atol=1e-13)
+    want = F.scaled_dot_product_attention(
+        torch.tensor(q).permute(1, 0, 2)[None], torch.tensor(k).permute(1, 0, 2)[None],
+        torch.tensor(v).permute(1, 0, 2)[None], enable_gqa=True)[0].permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_special_cases():
+    q = RNG.standard_normal((4, 2, 16))
+    k = RNG.standard_normal((9, 1, 16))
+    v = np.tile(RNG.standard_normal((1, 1, 16)), (9, 1, 1))     # every V row equal
+    np.testing.assert_allclose(oracle.gqa_attention(q, k, v), np.broadcast_to(v[0, 0], (4, 2, 16)),
+                               rtol=1e-13, atol=1e-14)
+    one = oracle.gqa_attention(q[:1], k[:1], RNG.standard_normal((1, 1, 16)))
+    assert one.shape == (1, 2, 16)
+    # a single key gets all the weight
+    vv = RNG.standard_normal((1, 1, 16))
+    np.testing.assert_allclose(oracle.gqa_attention(q, k[:1], vv), np.broadcast_to(vv[0, 0], (4, 2, 16)))
+
+
+# ----------------------------------------------------------------- linear / SwiGLU
+
+def test_linear_and_swiglu_vs_torch():
+    x = RNG.standard_normal((5, 24))
+    w = RNG.standard_normal((10, 24))
+    b = RNG.standard_normal(10)
+    np.testing.assert_allclose(oracle.linear(x, w, b),
+                               F.linear(torch.tensor(x), torch.tensor(w), torch.tensor(b)).numpy(),
+                               rtol=1e-12, atol=1e-12)
+    wg = RNG.standard_normal((7, 24))
+    wu = RNG.standard_normal((7, 24))
+    tx = torch.tensor(x)
+    want = (F.silu(F.linear(tx, torch.tensor(wg))) * F.linear(tx, torch.tensor(wu))).numpy()
+    np.testing.assert_allclose(oracle.swiglu(x, wg, wu), want, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- FP8 e4m3
+
+def test_e4m3_golden_table():
+    rows = []
+    with open(os.path.join(GOLDEN, "e4m3_codes.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                c, v = line.split()
+                rows.append((int(c, 16), float(v)))
+    for code, val in rows:
+        got = ofp8.e4m3_decode(np.array([code], np.uint8))[0]
+        if math.isnan(val):
+            assert math.isnan(got)
+        else:
+            assert got == val and math.copysign(1, got) == math.copysign(1, val), (hex(code), got, val)
+            assert ofp8.e4m3_encode(np.array([val]))[0] == code
+
+
+def test_e4m3_exhaustive_roundtrip_ties_saturation():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = ofp8.e4m3_decode(codes)
+    finite = ~np.isnan(vals)
+    assert finite.sum() == 254
+    assert np.array_equal(ofp8.e4m3_encode(vals[finite]), codes[finite])
+    # ties: the midpoint between neighbouring positive codes goes to the even mantissa
+    pos = np.arange(0, 0x7E)
+    lo, hi = ofp8.e4m3_decode(pos.astype(np.uint8)), ofp8.e4m3_decode((pos + 1).astype(np.uint8))
+    mid = (lo + hi) / 2
+    got = ofp8.e4m3_encode(mid).astype(int)
+    want = np.where(pos % 2 == 0, pos, pos + 1)
+    assert np.array_equal(got, want)
+    # just above / below a midpoint go to the nearer code
+    assert np.array_equal(ofp8.e4m3_encode(np.nextafter(mid, np.inf)).astype(int), pos + 1)
+    assert np.array_equal(ofp8.e4m3_encode(np.nextafter(mid, -np.inf)).astype(int), pos)
+    # saturation
+    big = np.array([448.0, 449.0, 464.0, 500.0, 1e6, np.inf, -1e9, -np.inf])
+    assert list(ofp8.e4m3_encode(big)) == [0x7E] * 6 + [0xFE] * 2
+    assert ofp8.e4m3_encode(np.array([np.nan]))[0] == 0x7F
+
+
+def test_e4m3_matches_torch_cast_in_range():
+    x = np.concatenate([RNG.standard_normal(20000) * s for s in (0.003, 0.1, 3, 60, 150)]).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    pos = np.arange(0, 0x7E)
+    mids = ((ofp8.e4m3_decode(pos.astype(np.uint8)) + ofp8.e4m3_decode((pos + 1).astype(np.uint8))) / 2)
+    x = np.concatenate([x, mids.astype(np.float32), -mids.astype(np.float32)])
+    want = torch.tensor(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ofp8.e4m3_encode(x), want)
+
+
+def test_rowwise_quantiser():
+    w = (RNG.standard_normal((6, 40)) * 0.02).astype(np.float32)
+    w[3] = 0.0
+    codes, scales = ofp8.quantize_rowwise_e4m3(w)
+    assert scales.dtype == np.float32 and scales[3] == 1.0
+    assert np.all(codes[3] == 0)
+    for o in (0, 1, 2, 4, 5):
+        i = np.argmax(np.abs(w[o]))
+        assert codes[o, i] in (0x7E, 0xFE)
+    deq = ofp8.dequantize_rowwise_e4m3(codes, scales)
+    # e4m3 keeps 3 mantissa bits: relative error of a normal value <= 2^-4
+    big = np.abs(w) > scales[:, None] * 2 ** -6
+    assert np.all(np.abs(deq - w)[big] <= np.abs(w)[big] * 2 ** -4 + 1e-12)
+
+
+# ----------------------------------------------------------------- layer / model composition
+
+MICRO = config("tiny", n_layers=2, hidden=64, n_q_heads=4, n_kv_heads=2, head_dim=16, inter=96,
+               n_prefix=7, action_dim=5, n_action_tokens=6, has_state_token=1, steps=3)
+
+
+def _layer_inputs(d, seed=0):
+    w = generate_weights(d, seed)
+    W = oracle.OracleWeights(w, d)
+    x = generate_inputs(d, seed)
+    lw = W.layer(0)
+    mod = oracle.adaln_table(lw["w_ada"], lw["b_ada"], 0.75, d.t_emb_dim)
+    kp = oracle.bf16_to_f64(x["k"][0, 0])
+    vp = oracle.bf16_to_f64(x["v"][0, 0])
+    h = RNG.standard_normal((d.ts, d.hidden)) * 0.1
+    pos = d.n_prefix + np.arange(d.ts, dtype=np.float64)
+    return W, lw, mod, kp, vp, h, pos
+
+
+def test_layer_zero_gates_is_identity():
+    d = MICRO
+    W, lw, mod, kp, vp, h, pos = _layer_inputs(d)
+    H = d.hidden
+    mod = mod.copy()
+    mod[2 * H:3 * H] = 0.0
+    mod[5 * H:6 * H] = 0.0
+    assert np.array_equal(oracle.dit_layer(h, lw, mod, kp, vp, pos, d), h)
+
+
+def test_layer_prefix_permutation_invariance():
+    d = MICRO
+    W, lw, mod, kp, vp, h, pos = _layer_inputs(d, seed=1)
+    perm = np.random.default_rng(9).permutation(kp.shape[0])
+    a = oracle.dit_layer(h, lw, mod, kp, vp, pos, d)
+    b = oracle.dit_layer(h, lw, mod, kp[perm], vp[perm], pos, d)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+    # swapping only K rows (not V) must change the result: the pairing of K and V matters
+    c = oracle.dit_layer(h, lw, mod, kp[perm], vp, pos, d)
+    assert np.max(np.abs(a - c)) > 1e-6
+
+
+def test_layer_trace_is_consistent():
+    d = MICRO
+    W, lw, mod, kp, vp, h, pos = _layer_inputs(d, seed=2)
+    tr = {}
+    out = oracle.dit_layer(h, lw, mod, kp, vp, pos, d, tr)
+    assert np.array_equal(out, tr["h_out"])
+    np.testing.assert_allclose(np.sqrt(np.mean(oracle.rms_norm(h, 0.0) ** 2, axis=1)), 1.0)
+    assert tr["q"].shape == (d.ts, d.n_q_heads, d.head_dim)
+    assert tr["m"].shape == (d.ts, d.inter)
+
+
+def test_batch_independence_bitwise_and_determinism():
+    d = MICRO.replace(batch=3)
+    w = generate_weights(d, 0)
+    x = generate_inputs(d, 0)
+    full = oracle.denoise_batch(w, x, d)
+    d1 = d.replace(batch=1)
+    for b in range(3):
+        xb = {k: v[b:b + 1] for k, v in x.items()}
+        one = oracle.denoise_batch(w, xb, d1)
+        assert np.array_equal(one[0], full[b])
+    again = oracle.denoise_batch(w, x, d)
+    assert np.array_equal(again, full)
+
+
+def test_single_step_is_one_euler_update():
+    d = MICRO
+    w = generate_weights(d, 0)
+    x = generate_inputs(d, 0)
+    W = oracle.OracleWeights(w, d)
+    noise = oracle.bf16_to_f64(x["noise"][0])
+    state = oracle.bf16_to_f64(x["state"][0])
+    kp, vp = oracle.bf16_to_f64(x["k"][0]), oracle.bf16_to_f64(x["v"][0])
+    v = oracle.velocity(noise, 1.0, state, W, kp, vp, d)
+    got = oracle.denoise(noise, state, W, kp, vp, d, 1)
+    assert np.array_equal(got, noise - v)
+
+
+# ----------------------------------------------------------------- input preparation
+
+def test_synth_bf16_rounding_matches_torch():
+    z = np.concatenate([RNG.standard_normal(50000).astype(np.float32) * s for s in (1e-3, 0.02, 1, 300)])
+    want = torch.tensor(z).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(f32_to_bf16_bits(z), want)
+    back = bf16_bits_to_f32(want)
+    assert np.array_equal(back, torch.tensor(z).to(torch.bfloat16).float().numpy())
+
+
+def test_layer_self_token_permutation_equivariance():
+    """No mask: permuting the self tokens together with their positions permutes the output."""
+    d = MICRO
+    W, lw, mod, kp, vp, h, pos = _layer_inputs(d, seed=3)
+    perm = np.array([4, 0, 6, 2, 1, 5, 3])[:d.ts]
+    a = oracle.dit_layer(h, lw, mod, kp, vp, pos, d)
+    b = oracle.dit_layer(h[perm], lw, mod, kp, vp, pos[perm], d)
+    np.testing.assert_allclose(b, a[perm], rtol=1e-12, atol=1e-13)
+
+
+def test_layer_branch_isolation_under_zero_gates():
+    """gate_a = 0 cuts the attention branch; gate_m = 0 cuts the MLP branch (adaLN-Zero)."""
+    d = MICRO
+    W, lw, mod, kp, vp, h, pos = _layer_inputs(d, seed=4)
+    H = d.hidden
+    rng = np.random.default_rng(11)
+
+    def perturbed(lw_, keys):
+        out = dict(lw_)
+        for k_ in keys:
+            out[k_] = lw_[k_] + rng.standard_normal(lw_[k_].shape) * 0.05
+        return out
+
+    m_a = mod.copy()
+    m_a[2 * H:3 * H] = 0.0                   # no attention branch
+    base = oracle.dit_layer(h, lw, m_a, kp, vp, pos, d)
+    alt = oracle.dit_layer(h, perturbed(lw, ("wq", "wk", "wv", "wo")), m_a,
+                           kp + 1.0, vp - 1.0, pos, d)
+    np.testing.assert_allclose(alt, base, rtol=1e-13, atol=1e-14)
+    m_a2 = m_a.copy()
+    m_a2[0:2 * H] += 0.3                     # attention shift/scale only feed that branch
+    np.testing.assert_allclose(oracle.dit_layer(h, lw, m_a2, kp, vp, pos, d), base, rtol=1e-13, atol=1e-14)
+
+    m_m = mod.copy()
+    m_m[5 * H:6 * H] = 0.0                   # no MLP branch
+    base = oracle.dit_layer(h, lw, m_m, kp, vp, pos, d)
+    alt = oracle.dit_layer(h, perturbed(lw, ("wg", "wu", "wd")), m_m, kp, vp, pos, d)
+    np.testing.assert_allclose(alt, base, rtol=1e-13, atol=1e-14)
+    m_m2 = m_m.copy()
+    m_m2[3 * H:5 * H] += 0.3
+    np.testing.assert_allclose(oracle.dit_layer(h, lw, m_m2, kp, vp, pos, d), base, rtol=1e-13, atol=1e-14)
+    # and each branch does contribute when its gate is on
+    assert np.max(np.abs(oracle.dit_layer(h, lw, mod, kp, vp, pos, d) - base)) > 1e-6
