@@ -1,0 +1,293 @@
+// Small kernels around the GEMMs: the per-step tail (final RMSNorm + adaLN modulate, action
+// out-projection, Euler update, next step's in-projection), the input-independent tables
+// (adaLN modulation per (step, layer), RoPE cos/sin for the self-token positions), weight
+// packing / fp8 quantisation at create time, and the prefix-cache layout at set_prefix time.
+#pragma once
+#include "ptx.cuh"
+
+namespace vla {
+
+constexpr int kTailThreads = 256;
+constexpr int kTileBytesPack = 16384;   // one packed weight tile (same as the GEMM's)
+constexpr int kMaxAction = 64;
+
+// ---------------------------------------------------------------- step tail / in-projection
+// One CTA per token row t = b * Ts + j.  Row j < has_state is the state token (not denoised),
+// the others are action tokens a = j - has_state.
+//  do_out: v = W_out (rms(h) * (1 + sc_f) + sh_f) + b_out ;  x += dt * v   (flow-matching Euler,
+//          "AI Infra如何优化VLA" section 整体方案)
+//  do_in : h = W_in x + b_in (state row: the cached W_st s + b_st), plus the row's sum of squares
+struct TailParams {
+  float* h;                 // [Ntok][H]
+  const float* ss;          // [ss_parts][Ntok]
+  int ss_parts;
+  float* ss_out;            // [1][Ntok]
+  const float* shift_f;     // [H]
+  const float* scale_f;     // [H]
+  const __nv_bfloat16* w_out;  // [A][H]
+  const __nv_bfloat16* b_out;  // [A]
+  const __nv_bfloat16* w_in;   // [H][A]
+  const __nv_bfloat16* b_in;   // [H]
+  const float* h_state0;    // [B][H]
+  const __nv_bfloat16* noise;  // [B][T][A] (init only)
+  float* x;                 // [B][T][A]
+  float* out;               // [B][T][A] copy of x after the update (or nullptr)
+  float* v_out;             // [B][T][A] velocity (debug, or nullptr)
+  float dt, eps;
+  int H, A, T, Ts, has_state, Ntok;
+  int do_out, do_in, init_from_noise;
+};
+
+__global__ void __launch_bounds__(kTailThreads) tail_kernel(const __grid_constant__ TailParams p) {
+  __shared__ float red[kTailThreads / 32][kMaxAction];
+  __shared__ float xs[kMaxAction];
+  __shared__ float rs_sh;
+  const int t = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = t / p.Ts, j = t % p.Ts;
+  const bool is_state = j < p.has_state;
+  const int a_row = j - p.has_state;
+  const int H = p.H, A = p.A;
+  pdl_trigger();
+  pdl_wait();
+  float* hrow = p.h + (size_t)t * H;
+  if (!is_state) {
+    float* xrow = p.x + ((size_t)b * p.T + a_row) * A;
+    if (p.init_from_noise) {
+      if (tid < A) xrow[tid] = __bfloat162float(p.noise[((size_t)b * p.T + a_row) * A + tid]);
+      __syncthreads();
+    }
+    if (p.do_out) {
+      if (tid == 0) {
+        float acc = 0.f;
+        for (int q = 0; q < p.ss_parts; ++q) acc += p.ss[(size_t)q * p.Ntok + t];
+        rs_sh = rsqrtf(acc / (float)H + p.eps);
+      }
+      __syncthreads();
+      const float rs = rs_sh;
+      float part[kMaxAction];
+      for (int a = 0; a < A; ++a) part[a] = 0.f;
+      for (int k = tid; k < H; k += kTailThreads) {
+        const float u = hrow[k] * rs * (1.f + p.scale_f[k]) + p.shift_f[k];
+        for (int a = 0; a < A; ++a) part[a] = fmaf(__bfloat162float(p.w_out[(size_t)a * H + k]), u, part[a]);
+      }
+      // fixed-order block reduction: warp shuffle tree, then warps in order
+      for (int a = 0; a < A; ++a) {
+        float v = part[a];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[warp][a] = v;
+      }
+      __syncthreads();
+      if (tid < A) {
+        float v = __bfloat162float(p.b_out[tid]);
+        for (int w = 0; w < kTailThreads / 32; ++w) v += red[w][tid];
+        if (p.v_out) p.v_out[((size_t)b * p.T + a_row) * A + tid] = v;
+        const float xn = xrow[tid] + p.dt * v;
+        xrow[tid] = xn;
+        if (p.out) p.out[((size_t)b * p.T + a_row) * A + tid] = xn;
+      }
+      __syncthreads();
+    }
+    if (p.do_in) {
+      if (tid < A) xs[tid] = xrow[tid];
+      __syncthreads();
+      float sq = 0.f;
+      for (int o = tid; o < H; o += kTailThreads) {
+        float v = __bfloat162float(p.b_in[o]);
+        for (int a = 0; a < A; ++a) v = fmaf(__bfloat162float(p.w_in[(size_t)o * A + a]), xs[a], v);
+        hrow[o] = v;
+        sq = fmaf(v, v, sq);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (lane == 0) red[warp][0] = sq;
+      __syncthreads();
+      if (tid == 0) {
+        float s = 0.f;
+        for (int w = 0; w < kTailThreads / 32; ++w) s += red[w][0];
+        p.ss_out[t] = s;
+      }
+    }
+  } else if (p.do_in) {
+    float sq = 0.f;
+    for (int o = tid; o < H; o += kTailThreads) {
+      const float v = p.h_state0[(size_t)b * H + o];
+      hrow[o] = v;
+      sq = fmaf(v, v, sq);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if (lane == 0) red[warp][0] = sq;
+    __syncthreads();
+    if (tid == 0) {
+      float s = 0.f;
+      for (int w = 0; w < kTailThreads / 32; ++w) s += red[w][0];
+      p.ss_out[t] = s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- input-independent tables
+// c_k = SiLU(temb(t_k)), temb(t) = [cos(a_i), sin(a_i)], a_i = 1000 t 10000^(-i/half), in double.
+__global__ void temb_kernel(double* c, int steps, int dt_dim) {
+  const int k = blockIdx.x, half = dt_dim / 2;
+  const double t = 1.0 - (double)k / (double)steps;
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double a = 1000.0 * t * exp(-log(10000.0) * (double)i / (double)half);
+    const double cs = cos(a), sn = sin(a);
+    c[(size_t)k * dt_dim + i] = cs / (1.0 + exp(-cs));
+    c[(size_t)k * dt_dim + half + i] = sn / (1.0 + exp(-sn));
+  }
+}
+
+// table[k][row] = W[row] . c_k + b[row] for rows of one adaLN weight (one warp per row).
+__global__ void adaln_table_kernel(const __nv_bfloat16* __restrict__ w, const __nv_bfloat16* __restrict__ bias,
+                                   const double* __restrict__ c, int rows, int dt_dim, int steps, float* out,
+                                   size_t step_stride) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  for (int k = 0; k < steps; ++k) {
+    double acc = 0.0;
+    for (int i = lane; i < dt_dim; i += 32) acc += (double)__bfloat162float(w[(size_t)row * dt_dim + i]) * c[(size_t)k * dt_dim + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) out[(size_t)k * step_stride + row] = (float)(acc + (double)__bfloat162float(bias[row]));
+  }
+}
+
+// rope[j][i] = (cos, sin)(theta), theta = (P + j) * base^(-2i/hd), in double.
+__global__ void rope_table_kernel(float2* rope, int Ts, int P, int hd, double base) {
+  const int half = hd / 2;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < Ts * half; e += gridDim.x * blockDim.x) {
+    const int j = e / half, i = e % half;
+    const double th = (double)(P + j) * pow(base, -2.0 * (double)i / (double)hd);
+    rope[e] = make_float2((float)cos(th), (float)sin(th));
+  }
+}
+
+// h_state0[b] = W_st s_b + b_st
+__global__ void state_proj_kernel(const __nv_bfloat16* w, const __nv_bfloat16* bias, const __nv_bfloat16* state,
+                                  float* out, int H, int A) {
+  const int b = blockIdx.y;
+  for (int o = blockIdx.x * blockDim.x + threadIdx.x; o < H; o += gridDim.x * blockDim.x) {
+    float v = __bfloat162float(bias[o]);
+    for (int a = 0; a < A; ++a)
+      v = fmaf(__bfloat162float(w[(size_t)o * A + a]), __bfloat162float(state[(size_t)b * A + a]), v);
+    out[(size_t)b * H + o] = v;
+  }
+}
+
+// ---------------------------------------------------------------- weight packing (create time)
+// Gather source rows (row pointers, nullptr = zero row) into 16 KB bf16 tiles [Mt][KB][128][64]
+// in the 128-byte swizzle layout.  One thread per 16-byte chunk.
+__global__ void pack_bf16_kernel(const __nv_bfloat16* const* __restrict__ rows, int K, int Mt, int KB,
+                                 uint8_t* __restrict__ dst) {
+  const size_t total = (size_t)Mt * KB * 128 * 8;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const int ch = (int)(e & 7);
+    const int r = (int)((e >> 3) & 127);
+    const size_t tile = e >> 10;
+    const int kb = (int)(tile % KB), mt = (int)(tile / KB);
+    const __nv_bfloat16* src = rows[mt * 128 + r];
+    const int k0 = kb * 64 + ch * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (src && k0 < K) v = *reinterpret_cast<const uint4*>(src + k0);
+    *reinterpret_cast<uint4*>(dst + tile * kTileBytesPack + sw128_chunk_byte(r, ch)) = v;
+  }
+}
+
+// Per-output-channel e4m3 quantisation (one warp per packed row):
+// scale = max|w| / 448 (IEEE division; 1 for a zero row), code = e4m3_rn_sat(w / scale).
+// Codes go to 16 KB tiles [Mt][KB8][128][128 B], 16-byte chunks swizzled like the bf16 tiles.
+__global__ void quant_e4m3_kernel(const __nv_bfloat16* const* __restrict__ rows, int K, int Mt, int KB8,
+                                  uint8_t* __restrict__ dst, float* __restrict__ scales) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= Mt * 128) return;
+  const __nv_bfloat16* src = rows[row];
+  float amax = 0.f;
+  if (src)
+    for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(__bfloat162float(src[k])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float sc = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+  if (lane == 0) scales[row] = sc;
+  const int mt = row >> 7, r = row & 127;
+  for (int c = lane; c < KB8 * 8; c += 32) {            // 16-element chunks along K
+    const int kb = c >> 3, ch = c & 7, k0 = c * 16;
+    uint32_t word[4] = {0, 0, 0, 0};
+    if (src) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int k = k0 + 2 * q;
+        const float lo = (k < K) ? __fdiv_rn(__bfloat162float(src[k]), sc) : 0.f;
+        const float hi = (k + 1 < K) ? __fdiv_rn(__bfloat162float(src[k + 1]), sc) : 0.f;
+        word[q >> 1] |= (uint32_t)f32x2_to_e4m3x2(lo, hi) << ((q & 1) * 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(dst + ((size_t)mt * KB8 + kb) * kTileBytesPack + sw128_chunk_byte(r, ch)) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+  }
+}
+
+// ---------------------------------------------------------------- prefix layout (set_prefix)
+// user K, V: [B][L][P][nkv][hd]  ->  K cache [L][B][nkv][Lpad][hd], V^T cache [L][B][nkv][hd][Lpad]
+__global__ void prefix_layout_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                                     __nv_bfloat16* kc, __nv_bfloat16* vct, int B, int L, int P, int nkv, int hd,
+                                     int Lpad) {
+  const size_t total = (size_t)B * L * P * nkv * hd;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const int d = (int)(e % hd);
+    size_t r = e / hd;
+    const int g = (int)(r % nkv); r /= nkv;
+    const int pp = (int)(r % P); r /= P;
+    const int l = (int)(r % L);
+    const int b = (int)(r / L);
+    const size_t cache = (((size_t)l * B + b) * nkv + g);
+    kc[(cache * Lpad + pp) * hd + d] = k[e];
+    vct[(cache * hd + d) * Lpad + pp] = v[e];
+  }
+}
+
+// ---------------------------------------------------------------- debug read-outs
+// ss[t] = sum_k h[t][k]^2 for one row per CTA (fixed-order block reduction)
+__global__ void row_sumsq_kernel(const float* h, float* ss, int H) {
+  __shared__ float red[32];
+  const int t = blockIdx.x, tid = threadIdx.x;
+  float s = 0.f;
+  for (int k = tid; k < H; k += blockDim.x) s = fmaf(h[(size_t)t * H + k], h[(size_t)t * H + k], s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((tid & 31) == 0) red[tid >> 5] = s;
+  __syncthreads();
+  if (tid == 0) {
+    float a = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) a += red[w];
+    ss[t] = a;
+  }
+}
+// swizzled operand tiles [Nt][KB][NT][64] -> fp32 [Ntok][K]
+__global__ void untile_kernel(const __nv_bfloat16* tiles, float* out, int Ntok, int K, int NT, int KB) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < Ntok * K; e += gridDim.x * blockDim.x) {
+    const int t = e / K, k = e % K;
+    const int nt = t / NT, row = t % NT;
+    out[e] = __bfloat162float(tiles[((size_t)nt * KB + (k >> 6)) * NT * 64 + sw128_elem_offset(row, k & 63)]);
+  }
+}
+__global__ void bf16_to_f32_kernel(const __nv_bfloat16* in, float* out, size_t n) {
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x)
+    out[e] = __bfloat162float(in[e]);
+}
+// self rows of the layer caches -> fp32 k [Ntok][nkv][hd], v [Ntok][nkv][hd]
+__global__ void self_kv_kernel(const __nv_bfloat16* kc, const __nv_bfloat16* vct, float* k, float* v, int B, int Ts,
+                               int nkv, int hd, int P, int Lpad) {
+  const int n = B * Ts * nkv * hd;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+    const int d = e % hd, g = (e / hd) % nkv, t = e / (hd * nkv);
+    const int b = t / Ts, j = t % Ts;
+    const size_t cache = (size_t)b * nkv + g;
+    k[e] = __bfloat162float(kc[(cache * Lpad + P + j) * hd + d]);
+    v[e] = __bfloat162float(vct[(cache * hd + d) * Lpad + P + j]);
+  }
+}
+
+}  // namespace vla

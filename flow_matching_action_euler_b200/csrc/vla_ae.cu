@@ -1,0 +1,940 @@
+// Host engine behind the C ABI in include/vla_ae.h.
+//
+// create:      plan every kernel of the loop (tiles, split-K cluster sizes, shared memory), allocate
+//              all device buffers once ("AI Infra如何优化VLA" section CUDA Graph: preallocate the
+//              buffers the captured graph uses), pack / quantise the weights.
+// set_prefix:  lay the VLM prefix K / V out for the attention kernel, project the state token,
+//              rebuild the RoPE table for the self-token positions.
+// denoise:     first call per step count builds the adaLN table and captures the whole N-step loop
+//              (1 + N * (5 L + 1) kernels chained by programmatic dependent launch) as one CUDA
+//              graph (same page and section: warm-up, capture, replay; APXInf article: capture once,
+//              replay every control cycle); later calls copy the noise in, replay, copy x out.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <vector>
+
+#include "../../include/vla_ae.h"
+#include "ptx.cuh"
+#include "gemm.cuh"
+#include "attention.cuh"
+#include "misc.cuh"
+
+using namespace vla;
+
+namespace {
+
+constexpr int kMaxDynSmem = 232448;      // 227 KB per CTA on sm_100
+constexpr int kGemmSmemBudget = 116 * 1024;  // leaves room for a second CTA per SM (PDL overlap)
+
+#define CK(call)                                                            \
+  do {                                                                      \
+    cudaError_t e_ = (call);                                                \
+    if (e_ != cudaSuccess) {                                                \
+      std::fprintf(stderr, "vla_ae: %s failed: %s (%s:%d)\n", #call,        \
+                   cudaGetErrorString(e_), __FILE__, __LINE__);             \
+      return e_ == cudaErrorMemoryAllocation ? VLA_AE_ENOMEM : VLA_AE_ECUDA; \
+    }                                                                       \
+  } while (0)
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+enum OpId { OP_QKV = 0, OP_O = 1, OP_GU = 2, OP_D = 3 };
+
+struct OpPlan {
+  int O = 0, K = 0, Mt = 0, KB = 0, KBt = 0, S = 1, stages = 1;
+  size_t wbytes = 0;        // packed tile bytes of one layer
+  size_t woff = 0;          // offset inside a layer's packed block
+  size_t soff = 0;          // offset of the op's scales inside a layer's scale block (floats)
+  int off_b = 0, off_conv = 0, off_bar = 0, smem = 0;
+};
+
+struct StepTables {
+  int steps = 0;
+  float* mod = nullptr;    // [steps][L][6H]
+  float* fmod = nullptr;   // [steps][2H]
+  cudaGraphExec_t exec = nullptr;
+  int captured_prefix = -1;
+};
+
+}  // namespace
+
+struct vla_ae {
+  vla_ae_dims d{};
+  int device = 0, num_sms = 148;
+  bool fp8 = false;
+  int Ts = 0, Ntok = 0, NT = 0, Nt = 0, qd = 0, kd = 0, Lpad = 0;
+  OpPlan op[4];
+  size_t layer_wbytes = 0, layer_scales = 0;
+  int attn_S = 1, attn_cmax = 0, attn_smem = 0;
+  AttnParams attn_proto{};
+  // device memory
+  std::vector<void*> allocs;
+  uint8_t* wpack = nullptr;
+  float* wscale = nullptr;
+  __nv_bfloat16 *w_in = nullptr, *b_in = nullptr, *w_st = nullptr, *b_st = nullptr, *w_out = nullptr,
+                *b_out = nullptr, *w_ada = nullptr, *b_ada = nullptr, *w_fada = nullptr, *b_fada = nullptr;
+  __nv_bfloat16 *kc = nullptr, *vct = nullptr, *q = nullptr, *act_o = nullptr, *act_m = nullptr,
+                *noise_stage = nullptr, *state_stage = nullptr;
+  float *h = nullptr, *ss = nullptr, *x = nullptr, *h_state0 = nullptr, *rope = nullptr, *out_stage = nullptr;
+  double* temb = nullptr;
+  unsigned* status = nullptr;
+  size_t device_bytes = 0;
+  int n_prefix = -1;
+  cudaStream_t cap = nullptr;
+  std::map<int, StepTables> tables;
+
+  template <typename T>
+  int alloc(T** p, size_t bytes) {
+    void* v = nullptr;
+    bytes = align_up(bytes ? bytes : 16, 256);
+    CK(cudaMalloc(&v, bytes));
+    allocs.push_back(v);
+    CK(cudaMemset(v, 0, bytes));
+    device_bytes += bytes;
+    *p = reinterpret_cast<T*>(v);
+    return VLA_AE_OK;
+  }
+  ~vla_ae() {
+    for (auto& kv : tables)
+      if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+    for (void* p : allocs) cudaFree(p);
+    if (cap) cudaStreamDestroy(cap);
+  }
+};
+
+namespace {
+
+// ------------------------------------------------------------------ launch helper
+template <typename Kern, typename Arg>
+cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x, bool pdl,
+                   const Arg& arg) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  int n = 0;
+  if (pdl) {
+    attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attrs[n].id = cudaLaunchAttributeClusterDimension;
+    attrs[n].val.clusterDim.x = cluster_x;
+    attrs[n].val.clusterDim.y = 1;
+    attrs[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, arg);
+}
+
+using GemmKernel = void (*)(const GemmParams);
+
+GemmKernel gemm_kernel_for(OpId id, bool fp8) {
+  switch (id) {
+    case OP_QKV: return fp8 ? gemm_stream_kernel<EPI_QKV, B_NORM, true> : gemm_stream_kernel<EPI_QKV, B_NORM, false>;
+    case OP_O: return fp8 ? gemm_stream_kernel<EPI_RESID, B_TILES, true> : gemm_stream_kernel<EPI_RESID, B_TILES, false>;
+    case OP_GU: return fp8 ? gemm_stream_kernel<EPI_SWIGLU, B_NORM, true> : gemm_stream_kernel<EPI_SWIGLU, B_NORM, false>;
+    default: return fp8 ? gemm_stream_kernel<EPI_RESID, B_TILES, true> : gemm_stream_kernel<EPI_RESID, B_TILES, false>;
+  }
+}
+
+using AttnKernel = void (*)(const AttnParams);
+AttnKernel attn_kernel_for(int hd) {
+  switch (hd) {
+    case 64: return attn_kernel<64>;
+    case 128: return attn_kernel<128>;
+    default: return attn_kernel<256>;
+  }
+}
+
+// shared-memory layout of one GEMM op for a given split / ring depth
+void gemm_layout(OpPlan& p, int NT, bool fp8) {
+  const int nkt_max = ceil_div(p.KBt, p.S);
+  const int nkb_max = std::min(nkt_max * (fp8 ? 2 : 1), p.KB);
+  const size_t a_region = std::max<size_t>((size_t)p.stages * kTileBytes, (size_t)NT * 128 * 4);
+  const size_t b_region = std::max<size_t>((size_t)nkb_max * NT * 128, (size_t)NT * 64 * 4);
+  const size_t conv = fp8 ? (size_t)kConvStages * 2 * kTileBytes : 0;
+  p.off_b = (int)a_region;
+  p.off_conv = (int)(a_region + b_region);
+  p.off_bar = (int)(a_region + b_region + conv);
+  const size_t bar_bytes = 8 * (2 * p.stages + 2 + 2 * kConvStages) + 16 + 4 * NT;
+  p.smem = (int)(p.off_bar + align_up(bar_bytes, 16) + 1024);   // + alignment slack
+}
+
+int plan_gemm(vla_ae* H, OpPlan& p, OpId id, int O, int K) {
+  const bool fp8 = H->fp8;
+  p.O = O;
+  p.K = K;
+  p.Mt = ceil_div(O, 128);
+  p.KB = ceil_div(K, 64);
+  p.KBt = fp8 ? ceil_div(K, 128) : p.KB;
+  p.wbytes = (size_t)p.Mt * p.KBt * kTileBytes;
+  const int ctas_per_split = p.Mt * H->Nt;
+  int S = std::max(1, std::min({16, p.KBt, H->num_sms / std::max(1, ctas_per_split)}));
+  GemmKernel kern = gemm_kernel_for(id, fp8);
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
+  for (; S >= 1; --S) {
+    p.S = S;
+    // ring depth: as deep as the budget allows (at least 2 when there is more than one tile)
+    const int nkt_max = ceil_div(p.KBt, S);
+    p.stages = 1;
+    gemm_layout(p, H->NT, fp8);
+    const int budget = fp8 ? kMaxDynSmem : kGemmSmemBudget;
+    while (p.stages < std::min(nkt_max, 8)) {
+      OpPlan t = p;
+      t.stages = p.stages + 1;
+      gemm_layout(t, H->NT, fp8);
+      if (t.smem > budget && p.stages >= 2) break;
+      if (t.smem > kMaxDynSmem) break;
+      p = t;
+    }
+    if (p.smem > kMaxDynSmem) continue;
+    if (S == 1) break;
+    // the grid must fit in one wave of co-resident clusters
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, p.Mt, H->Nt);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = p.smem;
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeClusterDimension;
+    a.val.clusterDim.x = S;
+    a.val.clusterDim.y = 1;
+    a.val.clusterDim.z = 1;
+    cfg.attrs = &a;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    if (nclusters >= ctas_per_split) break;
+  }
+  if (p.S < 1 || p.smem > kMaxDynSmem) return VLA_AE_EUNSUPPORTED;
+  return VLA_AE_OK;
+}
+
+// Which source matrix row feeds packed row `pr` of op `id` (matrix: 0 q,1 k,2 v,3 o,4 g,5 u,6 d; -1 pad).
+// QKV: each rotary pair (x_i, x_{i+hd/2}) of a q or k head becomes two adjacent packed rows so that
+// the epilogue can rotate it locally; v rows keep their order.  Gate/up rows are interleaved so
+// that SiLU(gate_j) * up_j is formed from two adjacent rows.
+void packed_row_source(const vla_ae* H, OpId id, int pr, int* matrix, int* row) {
+  const int hd = H->d.head_dim, half = hd / 2;
+  *matrix = -1;
+  *row = 0;
+  switch (id) {
+    case OP_QKV: {
+      if (pr < H->qd + H->kd) {
+        const bool isq = pr < H->qd;
+        const int local = isq ? pr : pr - H->qd;
+        const int head = local / hd, within = local % hd, i = within >> 1;
+        *matrix = isq ? 0 : 1;
+        *row = head * hd + i + ((within & 1) ? half : 0);
+      } else if (pr < H->qd + 2 * H->kd) {
+        *matrix = 2;
+        *row = pr - H->qd - H->kd;
+      }
+      break;
+    }
+    case OP_O:
+      if (pr < H->d.hidden) { *matrix = 3; *row = pr; }
+      break;
+    case OP_GU:
+      if (pr < 2 * H->d.inter) { *matrix = (pr & 1) ? 5 : 4; *row = pr >> 1; }
+      break;
+    case OP_D:
+      if (pr < H->d.hidden) { *matrix = 6; *row = pr; }
+      break;
+  }
+}
+
+int validate_dims(const vla_ae_dims* d) {
+  if (!d) return VLA_AE_EINVAL;
+  if (d->n_layers < 1 || d->hidden < 8 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->head_dim < 2 ||
+      d->inter < 8 || d->t_emb_dim < 2 || d->action_dim < 1 || d->n_action_tokens < 1 || d->max_prefix < 0 ||
+      d->batch < 1)
+    return VLA_AE_EINVAL;
+  if (d->has_state_token != 0 && d->has_state_token != 1) return VLA_AE_EINVAL;
+  if (d->hidden % 8 || d->inter % 8 || d->t_emb_dim % 2 || d->n_q_heads % d->n_kv_heads) return VLA_AE_EINVAL;
+  if (d->action_dim > kMaxAction) return VLA_AE_EINVAL;
+  if ((long long)d->batch * (d->n_action_tokens + d->has_state_token) > 4096) return VLA_AE_EINVAL;
+  if (!(d->rope_theta > 0.f) || !(d->rms_eps >= 0.f)) return VLA_AE_EINVAL;
+  if (d->wtype != VLA_AE_BF16 && d->wtype != VLA_AE_FP8_E4M3) return VLA_AE_EINVAL;
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return VLA_AE_EUNSUPPORTED;
+  return VLA_AE_OK;
+}
+
+// ------------------------------------------------------------------ attention plan
+int plan_attention(vla_ae* H, int P) {
+  const int L = P + H->Ts;
+  const int hd = H->d.head_dim;
+  const int groups = H->d.n_q_heads * H->d.batch;
+  int S = std::max(1, std::min({16, L, H->num_sms / std::max(1, groups)}));
+  AttnKernel kern = attn_kernel_for(hd);
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
+  // candidate cluster sizes: the preferred one, then smaller, then larger (more, shorter chunks)
+  std::vector<int> cands;
+  for (int c = S; c >= 1; --c) cands.push_back(c);
+  for (int c = S + 1; c <= std::min(16, L); ++c) cands.push_back(c);
+  for (int S : cands) {
+    const int cmax = ceil_div(L, S);
+    const int Ts = H->Ts;
+    size_t off = (size_t)Ts * hd * 4;
+    AttnParams a{};
+    a.off_k = (int)off;
+    off = align_up(off + (size_t)cmax * (hd + 2) * 2, 16);
+    a.off_v = (int)off;
+    off = align_up(off + (size_t)hd * (cmax + 2) * 2, 16);
+    a.off_s = (int)off;
+    off = align_up(off + (size_t)Ts * cmax * 4, 16);
+    a.off_o = (int)off;
+    off = align_up(off + (size_t)Ts * hd * 4, 16);
+    a.off_ml = (int)off;
+    off += (size_t)(2 + 16) * Ts * 4;
+    a.smem_bytes = (int)off;
+    if (off > (size_t)kMaxDynSmem) continue;
+    if (S > 1) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(S, H->d.n_q_heads, H->d.batch);
+      cfg.blockDim = dim3(kAttnThreads);
+      cfg.dynamicSmemBytes = off;
+      cudaLaunchAttribute at;
+      at.id = cudaLaunchAttributeClusterDimension;
+      at.val.clusterDim.x = S;
+      at.val.clusterDim.y = 1;
+      at.val.clusterDim.z = 1;
+      cfg.attrs = &at;
+      cfg.numAttrs = 1;
+      int ncl = 0;
+      if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      if (ncl < 1) continue;
+    }
+    H->attn_S = S;
+    H->attn_cmax = cmax;
+    H->attn_smem = (int)off;
+    H->attn_proto = a;
+    return VLA_AE_OK;
+  }
+  return VLA_AE_EUNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ per-op launch
+struct LayerPtrs {
+  const float *shift_a, *scale_a, *gate_a, *shift_m, *scale_m, *gate_m;
+};
+
+LayerPtrs layer_mod(const vla_ae* H, const StepTables& T, int step, int layer) {
+  const size_t Hd = H->d.hidden;
+  const float* base = T.mod + ((size_t)step * H->d.n_layers + layer) * 6 * Hd;
+  return {base, base + Hd, base + 2 * Hd, base + 3 * Hd, base + 4 * Hd, base + 5 * Hd};
+}
+
+GemmParams gemm_common(const vla_ae* H, OpId id, int layer) {
+  const OpPlan& p = H->op[id];
+  GemmParams g{};
+  g.w = H->wpack + (size_t)layer * H->layer_wbytes + p.woff;
+  g.wscale = H->fp8 ? H->wscale + (size_t)layer * H->layer_scales + p.soff : nullptr;
+  g.Mt = p.Mt;
+  g.KBt = p.KBt;
+  g.K = p.K;
+  g.S = p.S;
+  g.stages = p.stages;
+  g.Ntok = H->Ntok;
+  g.NT = H->NT;
+  g.KB = p.KB;
+  g.O = p.O;
+  g.eps = H->d.rms_eps;
+  g.status = H->status;
+  g.off_b = p.off_b;
+  g.off_conv = p.off_conv;
+  g.off_bar = p.off_bar;
+  g.smem_bytes = p.smem;
+  return g;
+}
+
+cudaError_t launch_gemm(const vla_ae* H, OpId id, const GemmParams& g, cudaStream_t st) {
+  const OpPlan& p = H->op[id];
+  return launch(gemm_kernel_for(id, H->fp8), dim3(p.S, p.Mt, H->Nt), dim3(kGemmThreads), p.smem, st, p.S, true, g);
+}
+
+int ss_parts_of(const vla_ae* H, OpId id) { return H->op[id].Mt * H->op[id].S; }
+
+// The five kernels of one DiT layer.  `ss_in_parts`: partial sums of squares feeding the first norm.
+cudaError_t enqueue_layer(vla_ae* H, const StepTables& T, int step, int layer, int ss_in_parts, cudaStream_t st,
+                          const vla_ae_trace* trace) {
+  const vla_ae_dims& d = H->d;
+  const LayerPtrs m = layer_mod(H, T, step, layer);
+  const size_t cache = (size_t)layer * d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+  cudaError_t e;
+  {  // RMSNorm + modulate -> QKV -> RoPE -> q, K/V caches
+    GemmParams g = gemm_common(H, OP_QKV, layer);
+    g.h = H->h;
+    g.ss = H->ss;
+    g.ss_parts = ss_in_parts;
+    g.shift = m.shift_a;
+    g.scale = m.scale_a;
+    g.q_out = H->q;
+    g.kc = H->kc + cache;
+    g.vct = H->vct + cache;
+    g.rope = H->rope;
+    g.nq = d.n_q_heads;
+    g.nkv = d.n_kv_heads;
+    g.hd = d.head_dim;
+    g.Ts = H->Ts;
+    g.P = H->n_prefix;
+    g.Lpad = H->Lpad;
+    if ((e = launch_gemm(H, OP_QKV, g, st)) != cudaSuccess) return e;
+  }
+  if (trace && (trace->q || trace->k || trace->v)) {
+    if (trace->q) bf16_to_f32_kernel<<<64, 256, 0, st>>>(H->q, trace->q, (size_t)H->Ntok * H->qd);
+    if (trace->k && trace->v)
+      self_kv_kernel<<<64, 256, 0, st>>>(H->kc + cache, H->vct + cache, trace->k, trace->v, d.batch, H->Ts,
+                                         d.n_kv_heads, d.head_dim, H->n_prefix, H->Lpad);
+  }
+  {  // attention over prefix + self
+    AttnParams a = H->attn_proto;
+    a.q = H->q;
+    a.kc = H->kc + cache;
+    a.vct = H->vct + cache;
+    a.o_tiles = H->act_o;
+    a.nq = d.n_q_heads;
+    a.nkv = d.n_kv_heads;
+    a.hd = d.head_dim;
+    a.Ts = H->Ts;
+    a.P = H->n_prefix;
+    a.Lpad = H->Lpad;
+    a.Ntok = H->Ntok;
+    a.NT = H->NT;
+    a.KBo = H->op[OP_O].KB;
+    a.S = H->attn_S;
+    a.cmax = H->attn_cmax;
+    a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
+    if ((e = launch(attn_kernel_for(d.head_dim), dim3(H->attn_S, d.n_q_heads, d.batch), dim3(kAttnThreads),
+                    H->attn_smem, st, H->attn_S, true, a)) != cudaSuccess)
+      return e;
+  }
+  if (trace && trace->o) untile_kernel<<<64, 256, 0, st>>>(H->act_o, trace->o, H->Ntok, H->qd, H->NT, H->op[OP_O].KB);
+  {  // o-projection + gated residual
+    GemmParams g = gemm_common(H, OP_O, layer);
+    g.act = H->act_o;
+    g.h_out = H->h;
+    g.gate = m.gate_a;
+    g.ss_out = H->ss;
+    if ((e = launch_gemm(H, OP_O, g, st)) != cudaSuccess) return e;
+  }
+  if (trace && trace->h_attn)
+    cudaMemcpyAsync(trace->h_attn, H->h, (size_t)H->Ntok * d.hidden * 4, cudaMemcpyDeviceToDevice, st);
+  {  // RMSNorm + modulate -> gate/up -> SwiGLU
+    GemmParams g = gemm_common(H, OP_GU, layer);
+    g.h = H->h;
+    g.ss = H->ss;
+    g.ss_parts = ss_parts_of(H, OP_O);
+    g.shift = m.shift_m;
+    g.scale = m.scale_m;
+    g.m_out = H->act_m;
+    g.KBm = H->op[OP_D].KB;
+    if ((e = launch_gemm(H, OP_GU, g, st)) != cudaSuccess) return e;
+  }
+  if (trace && trace->m) untile_kernel<<<64, 256, 0, st>>>(H->act_m, trace->m, H->Ntok, d.inter, H->NT, H->op[OP_D].KB);
+  {  // down-projection + gated residual
+    GemmParams g = gemm_common(H, OP_D, layer);
+    g.act = H->act_m;
+    g.h_out = H->h;
+    g.gate = m.gate_m;
+    g.ss_out = H->ss;
+    if ((e = launch_gemm(H, OP_D, g, st)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+TailParams tail_common(const vla_ae* H) {
+  TailParams t{};
+  t.h = H->h;
+  t.ss = H->ss;
+  t.ss_out = H->ss;
+  t.w_out = H->w_out;
+  t.b_out = H->b_out;
+  t.w_in = H->w_in;
+  t.b_in = H->b_in;
+  t.h_state0 = H->h_state0;
+  t.noise = H->noise_stage;
+  t.x = H->x;
+  t.eps = H->d.rms_eps;
+  t.H = H->d.hidden;
+  t.A = H->d.action_dim;
+  t.T = H->d.n_action_tokens;
+  t.Ts = H->Ts;
+  t.has_state = H->d.has_state_token;
+  t.Ntok = H->Ntok;
+  return t;
+}
+
+cudaError_t launch_tail(const vla_ae* H, const TailParams& t, cudaStream_t st) {
+  return launch(tail_kernel, dim3(H->Ntok), dim3(kTailThreads), 0, st, 1, true, t);
+}
+
+// The whole N-step loop (what the graph holds).
+cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
+  const int N = T.steps, L = H->d.n_layers;
+  TailParams t0 = tail_common(H);
+  t0.init_from_noise = 1;
+  t0.do_in = 1;
+  cudaError_t e;
+  if ((e = launch_tail(H, t0, st)) != cudaSuccess) return e;
+  for (int k = 0; k < N; ++k) {
+    for (int l = 0; l < L; ++l) {
+      const int parts = l == 0 ? 1 : ss_parts_of(H, OP_D);
+      if ((e = enqueue_layer(H, T, k, l, parts, st, nullptr)) != cudaSuccess) return e;
+    }
+    TailParams t = tail_common(H);
+    t.ss_parts = ss_parts_of(H, OP_D);
+    t.shift_f = T.fmod + (size_t)k * 2 * H->d.hidden;
+    t.scale_f = t.shift_f + H->d.hidden;
+    t.dt = -1.0f / (float)N;
+    t.do_out = 1;
+    t.do_in = k + 1 < N;
+    t.out = k + 1 == N ? H->out_stage : nullptr;
+    if ((e = launch_tail(H, t, st)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+int get_tables(vla_ae* H, int steps, StepTables** out) {
+  auto it = H->tables.find(steps);
+  if (it != H->tables.end()) {
+    *out = &it->second;
+    return VLA_AE_OK;
+  }
+  StepTables T;
+  T.steps = steps;
+  const vla_ae_dims& d = H->d;
+  const size_t Hd = d.hidden;
+  int rc;
+  if ((rc = H->alloc(&T.mod, (size_t)steps * d.n_layers * 6 * Hd * 4))) return rc;
+  if ((rc = H->alloc(&T.fmod, (size_t)steps * 2 * Hd * 4))) return rc;
+  double* c = nullptr;
+  CK(cudaMalloc(&c, (size_t)steps * d.t_emb_dim * sizeof(double)));
+  temb_kernel<<<steps, 128, 0, H->cap>>>(c, steps, d.t_emb_dim);
+  for (int l = 0; l < d.n_layers; ++l) {
+    const int rows = 6 * d.hidden;
+    adaln_table_kernel<<<ceil_div(rows, 8), 256, 0, H->cap>>>(H->w_ada + (size_t)l * rows * d.t_emb_dim,
+                                                                H->b_ada + (size_t)l * rows, c, rows, d.t_emb_dim,
+                                                                steps, T.mod + (size_t)l * rows,
+                                                                (size_t)d.n_layers * rows);
+  }
+  adaln_table_kernel<<<ceil_div(2 * d.hidden, 8), 256, 0, H->cap>>>(H->w_fada, H->b_fada, c, 2 * d.hidden,
+                                                                     d.t_emb_dim, steps, T.fmod, 2 * Hd);
+  CK(cudaGetLastError());
+  CK(cudaStreamSynchronize(H->cap));
+  CK(cudaFree(c));
+  auto res = H->tables.emplace(steps, T);
+  *out = &res.first->second;
+  return VLA_AE_OK;
+}
+
+int ensure_graph(vla_ae* H, StepTables* T) {
+  if (T->exec && T->captured_prefix == H->n_prefix) return VLA_AE_OK;
+  if (T->exec) {
+    cudaGraphExecDestroy(T->exec);
+    T->exec = nullptr;
+  }
+  cudaGraph_t g = nullptr;
+  CK(cudaStreamBeginCapture(H->cap, cudaStreamCaptureModeThreadLocal));
+  cudaError_t e = enqueue_loop(H, *T, H->cap);
+  cudaError_t e2 = cudaStreamEndCapture(H->cap, &g);
+  if (e != cudaSuccess || e2 != cudaSuccess) {
+    std::fprintf(stderr, "vla_ae: graph capture failed: %s / %s\n", cudaGetErrorString(e), cudaGetErrorString(e2));
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return VLA_AE_ECUDA;
+  }
+  CK(cudaGraphInstantiate(&T->exec, g, 0));
+  cudaGraphDestroy(g);
+  T->captured_prefix = H->n_prefix;
+  return VLA_AE_OK;
+}
+
+// copy a bf16 blob (host or device) to a fresh device buffer owned by H
+int upload_bf16(vla_ae* H, __nv_bfloat16** dst, const void* src, size_t n, int on_device) {
+  int rc = H->alloc(dst, n * 2);
+  if (rc) return rc;
+  if (!src) return VLA_AE_EINVAL;
+  CK(cudaMemcpy(*dst, src, n * 2, on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice));
+  return VLA_AE_OK;
+}
+
+int pack_weights(vla_ae* H, const vla_ae_weights* w) {
+  const vla_ae_dims& d = H->d;
+  const int Hd = d.hidden, I = d.inter;
+  const size_t sizes[7] = {(size_t)H->qd * Hd, (size_t)H->kd * Hd, (size_t)H->kd * Hd, (size_t)Hd * H->qd,
+                           (size_t)I * Hd,     (size_t)I * Hd,     (size_t)Hd * I};
+  const int ldk[7] = {Hd, Hd, Hd, H->qd, Hd, Hd, I};
+  __nv_bfloat16* stage[7] = {};
+  for (int i = 0; i < 7; ++i) CK(cudaMalloc(&stage[i], sizes[i] * 2));
+  int maxrows = 0;
+  for (int id = 0; id < 4; ++id) maxrows = std::max(maxrows, H->op[id].Mt * 128);
+  const __nv_bfloat16** rowptr_dev = nullptr;
+  CK(cudaMalloc(&rowptr_dev, (size_t)maxrows * sizeof(void*)));
+  std::vector<const __nv_bfloat16*> rows(maxrows);
+  const void* const* src_arrays[7] = {w->wq, w->wk, w->wv, w->wo, w->wg, w->wu, w->wd};
+  int rc = VLA_AE_OK;
+  for (int l = 0; l < d.n_layers && rc == VLA_AE_OK; ++l) {
+    const __nv_bfloat16* src[7];
+    for (int i = 0; i < 7; ++i) {
+      if (!src_arrays[i] || !src_arrays[i][l]) { rc = VLA_AE_EINVAL; break; }
+      if (w->on_device) {
+        src[i] = reinterpret_cast<const __nv_bfloat16*>(src_arrays[i][l]);
+      } else {
+        CK(cudaMemcpy(stage[i], src_arrays[i][l], sizes[i] * 2, cudaMemcpyHostToDevice));
+        src[i] = stage[i];
+      }
+    }
+    if (rc) break;
+    for (int id = 0; id < 4; ++id) {
+      const OpPlan& p = H->op[id];
+      for (int pr = 0; pr < p.Mt * 128; ++pr) {
+        int mat, row;
+        packed_row_source(H, (OpId)id, pr, &mat, &row);
+        rows[pr] = mat < 0 ? nullptr : src[mat] + (size_t)row * ldk[mat];
+      }
+      CK(cudaMemcpy(rowptr_dev, rows.data(), (size_t)p.Mt * 128 * sizeof(void*), cudaMemcpyHostToDevice));
+      uint8_t* dst = H->wpack + (size_t)l * H->layer_wbytes + p.woff;
+      if (H->fp8) {
+        quant_e4m3_kernel<<<ceil_div(p.Mt * 128, 8), 256>>>(rowptr_dev, p.K, p.Mt, p.KBt, dst,
+                                                           H->wscale + (size_t)l * H->layer_scales + p.soff);
+      } else {
+        pack_bf16_kernel<<<1024, 256>>>(rowptr_dev, p.K, p.Mt, p.KB, dst);
+      }
+      CK(cudaGetLastError());
+      CK(cudaDeviceSynchronize());   // rows[] and the staging buffers are reused
+    }
+  }
+  for (int i = 0; i < 7; ++i) cudaFree(stage[i]);
+  cudaFree(rowptr_dev);
+  return rc;
+}
+
+int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
+  int rc;
+  H->d = *dims;
+  const vla_ae_dims& d = H->d;
+  H->fp8 = d.wtype == VLA_AE_FP8_E4M3;
+  CK(cudaGetDevice(&H->device));
+  CK(cudaDeviceGetAttribute(&H->num_sms, cudaDevAttrMultiProcessorCount, H->device));
+  int major = 0;
+  CK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, H->device));
+  if (major != 10) return VLA_AE_EUNSUPPORTED;
+  CK(cudaStreamCreateWithFlags(&H->cap, cudaStreamNonBlocking));
+  H->Ts = d.n_action_tokens + d.has_state_token;
+  H->Ntok = d.batch * H->Ts;
+  H->Nt = ceil_div(H->Ntok, 256);
+  H->NT = (int)align_up(ceil_div(H->Ntok, H->Nt), 32);
+  H->qd = d.n_q_heads * d.head_dim;
+  H->kd = d.n_kv_heads * d.head_dim;
+  H->Lpad = (int)align_up((size_t)d.max_prefix + H->Ts, 8);
+  if ((rc = plan_gemm(H, H->op[OP_QKV], OP_QKV, H->qd + 2 * H->kd, d.hidden))) return rc;
+  if ((rc = plan_gemm(H, H->op[OP_O], OP_O, d.hidden, H->qd))) return rc;
+  if ((rc = plan_gemm(H, H->op[OP_GU], OP_GU, 2 * d.inter, d.hidden))) return rc;
+  if ((rc = plan_gemm(H, H->op[OP_D], OP_D, d.hidden, d.inter))) return rc;
+  size_t woff = 0, soff = 0;
+  for (int id = 0; id < 4; ++id) {
+    H->op[id].woff = woff;
+    H->op[id].soff = soff;
+    woff += H->op[id].wbytes;
+    soff += (size_t)H->op[id].Mt * 128;
+  }
+  H->layer_wbytes = woff;
+  H->layer_scales = soff;
+  if ((rc = plan_attention(H, d.max_prefix))) return rc;
+
+  const size_t L = d.n_layers, Hd = d.hidden, A = d.action_dim, B = d.batch;
+  if ((rc = H->alloc(&H->wpack, L * H->layer_wbytes))) return rc;
+  if (H->fp8 && (rc = H->alloc(&H->wscale, L * H->layer_scales * 4))) return rc;
+  if ((rc = H->alloc(&H->status, 16))) return rc;
+  const size_t cache = L * B * d.n_kv_heads * (size_t)H->Lpad * d.head_dim;
+  if ((rc = H->alloc(&H->kc, cache * 2))) return rc;
+  if ((rc = H->alloc(&H->vct, cache * 2))) return rc;
+  if ((rc = H->alloc(&H->q, (size_t)H->Ntok * H->qd * 2))) return rc;
+  if ((rc = H->alloc(&H->act_o, (size_t)H->Nt * H->op[OP_O].KB * H->NT * 64 * 2))) return rc;
+  if ((rc = H->alloc(&H->act_m, (size_t)H->Nt * H->op[OP_D].KB * H->NT * 64 * 2))) return rc;
+  if ((rc = H->alloc(&H->noise_stage, B * d.n_action_tokens * A * 2))) return rc;
+  if ((rc = H->alloc(&H->state_stage, B * A * 2))) return rc;
+  if ((rc = H->alloc(&H->h, (size_t)H->Ntok * Hd * 4))) return rc;
+  const int parts = std::max({1, ss_parts_of(H, OP_O), ss_parts_of(H, OP_D)});
+  if ((rc = H->alloc(&H->ss, (size_t)parts * H->Ntok * 4))) return rc;
+  if ((rc = H->alloc(&H->x, B * d.n_action_tokens * A * 4))) return rc;
+  if ((rc = H->alloc(&H->out_stage, B * d.n_action_tokens * A * 4))) return rc;
+  if ((rc = H->alloc(&H->h_state0, B * Hd * 4))) return rc;
+  if ((rc = H->alloc(&H->rope, (size_t)H->Ts * (d.head_dim / 2) * 8))) return rc;
+
+  if (!w) return VLA_AE_EINVAL;
+  const int od = w->on_device;
+  if (od) {  // device matrices are read in 16-byte vectors
+    const void* const* arrays[7] = {w->wq, w->wk, w->wv, w->wo, w->wg, w->wu, w->wd};
+    for (int i = 0; i < 7; ++i)
+      for (size_t l = 0; arrays[i] && l < (size_t)d.n_layers; ++l)
+        if (reinterpret_cast<uintptr_t>(arrays[i][l]) % 16) return VLA_AE_EINVAL;
+  }
+  if ((rc = upload_bf16(H, &H->w_in, w->w_in, Hd * A, od))) return rc;
+  if ((rc = upload_bf16(H, &H->b_in, w->b_in, Hd, od))) return rc;
+  if (d.has_state_token) {
+    if ((rc = upload_bf16(H, &H->w_st, w->w_state, Hd * A, od))) return rc;
+    if ((rc = upload_bf16(H, &H->b_st, w->b_state, Hd, od))) return rc;
+  }
+  if ((rc = upload_bf16(H, &H->w_out, w->w_out, A * Hd, od))) return rc;
+  if ((rc = upload_bf16(H, &H->b_out, w->b_out, A, od))) return rc;
+  if ((rc = upload_bf16(H, &H->w_fada, w->w_fada, 2 * Hd * d.t_emb_dim, od))) return rc;
+  if ((rc = upload_bf16(H, &H->b_fada, w->b_fada, 2 * Hd, od))) return rc;
+  if (!w->w_ada || !w->b_ada) return VLA_AE_EINVAL;
+  if ((rc = H->alloc(&H->w_ada, L * 6 * Hd * d.t_emb_dim * 2))) return rc;
+  if ((rc = H->alloc(&H->b_ada, L * 6 * Hd * 2))) return rc;
+  for (size_t l = 0; l < L; ++l) {
+    if (!w->w_ada[l] || !w->b_ada[l]) return VLA_AE_EINVAL;
+    const cudaMemcpyKind kind = od ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    CK(cudaMemcpy(H->w_ada + l * 6 * Hd * d.t_emb_dim, w->w_ada[l], 6 * Hd * d.t_emb_dim * 2, kind));
+    CK(cudaMemcpy(H->b_ada + l * 6 * Hd, w->b_ada[l], 6 * Hd * 2, kind));
+  }
+  if ((rc = pack_weights(H, w))) return rc;
+  CK(cudaDeviceSynchronize());
+  return VLA_AE_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* vla_ae_strerror(int code) {
+  switch (code) {
+    case VLA_AE_OK: return "ok";
+    case VLA_AE_EINVAL: return "invalid argument";
+    case VLA_AE_ENOMEM: return "out of device memory";
+    case VLA_AE_ECUDA: return "CUDA error";
+    case VLA_AE_ENOPREFIX: return "prefix not set";
+    case VLA_AE_ETIMEOUT: return "device-side wait timed out";
+    case VLA_AE_EUNSUPPORTED: return "unsupported configuration";
+    default: return "unknown error";
+  }
+}
+
+int vla_ae_create(const vla_ae_dims* dims, const vla_ae_weights* weights, vla_ae_t* out) {
+  if (!out) return VLA_AE_EINVAL;
+  *out = nullptr;
+  int rc = validate_dims(dims);
+  if (rc) return rc;
+  if (!weights) return VLA_AE_EINVAL;
+  auto H = std::make_unique<vla_ae>();
+  rc = create_impl(dims, weights, H.get());
+  if (rc) return rc;
+  *out = H.release();
+  return VLA_AE_OK;
+}
+
+void vla_ae_destroy(vla_ae_t h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  delete h;
+}
+
+int vla_ae_set_prefix(vla_ae_t H, const void* k, const void* v, int n_prefix, const void* state, int on_device,
+                      void* stream) {
+  if (!H || n_prefix < 0 || n_prefix > H->d.max_prefix) return VLA_AE_EINVAL;
+  if (n_prefix > 0 && (!k || !v)) return VLA_AE_EINVAL;
+  if (H->d.has_state_token && !state) return VLA_AE_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const vla_ae_dims& d = H->d;
+  if (n_prefix != H->n_prefix) {
+    int rc = plan_attention(H, n_prefix);
+    if (rc) return rc;
+  }
+  const size_t n = (size_t)d.batch * d.n_layers * n_prefix * d.n_kv_heads * d.head_dim;
+  if (n > 0) {
+    const __nv_bfloat16 *kd = reinterpret_cast<const __nv_bfloat16*>(k), *vd = reinterpret_cast<const __nv_bfloat16*>(v);
+    __nv_bfloat16 *kt = nullptr, *vt = nullptr;
+    if (!on_device) {
+      CK(cudaMallocAsync(&kt, n * 2, st));
+      CK(cudaMallocAsync(&vt, n * 2, st));
+      CK(cudaMemcpyAsync(kt, k, n * 2, cudaMemcpyHostToDevice, st));
+      CK(cudaMemcpyAsync(vt, v, n * 2, cudaMemcpyHostToDevice, st));
+      kd = kt;
+      vd = vt;
+    }
+    prefix_layout_kernel<<<4 * H->num_sms, 256, 0, st>>>(kd, vd, H->kc, H->vct, d.batch, d.n_layers, n_prefix,
+                                                         d.n_kv_heads, d.head_dim, H->Lpad);
+    CK(cudaGetLastError());
+    if (kt) CK(cudaFreeAsync(kt, st));
+    if (vt) CK(cudaFreeAsync(vt, st));
+  }
+  if (d.has_state_token) {
+    CK(cudaMemcpyAsync(H->state_stage, state, (size_t)d.batch * d.action_dim * 2,
+                       on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, st));
+    state_proj_kernel<<<dim3(ceil_div(d.hidden, 256), d.batch), 256, 0, st>>>(H->w_st, H->b_st, H->state_stage,
+                                                                               H->h_state0, d.hidden, d.action_dim);
+  }
+  rope_table_kernel<<<ceil_div(H->Ts * d.head_dim / 2, 256), 256, 0, st>>>(reinterpret_cast<float2*>(H->rope), H->Ts,
+                                                                           n_prefix, d.head_dim, (double)d.rope_theta);
+  CK(cudaGetLastError());
+  H->n_prefix = n_prefix;
+  return VLA_AE_OK;
+}
+
+static int denoise_common(vla_ae_t H, const void* noise, int steps, float* out, void* stream, bool host) {
+  if (!H || !noise || !out || steps < 1) return VLA_AE_EINVAL;
+  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  StepTables* T = nullptr;
+  int rc = get_tables(H, steps, &T);
+  if (rc) return rc;
+  if ((rc = ensure_graph(H, T))) return rc;
+  const vla_ae_dims& d = H->d;
+  const size_t nx = (size_t)d.batch * d.n_action_tokens * d.action_dim;
+  CK(cudaMemcpyAsync(H->noise_stage, noise, nx * 2, host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
+  CK(cudaGraphLaunch(T->exec, st));
+  CK(cudaMemcpyAsync(out, H->out_stage, nx * 4, host ? cudaMemcpyDeviceToHost : cudaMemcpyDeviceToDevice, st));
+  return VLA_AE_OK;
+}
+
+int vla_ae_denoise(vla_ae_t H, const void* noise, int steps, float* out, void* stream) {
+  return denoise_common(H, noise, steps, out, stream, false);
+}
+
+int vla_ae_denoise_host(vla_ae_t H, const void* noise_host, int steps, float* out_host, void* stream) {
+  return denoise_common(H, noise_host, steps, out_host, stream, true);
+}
+
+int vla_ae_status(vla_ae_t H) {
+  if (!H) return VLA_AE_EINVAL;
+  CK(cudaDeviceSynchronize());
+  unsigned s = 0;
+  CK(cudaMemcpy(&s, H->status, 4, cudaMemcpyDeviceToHost));
+  CK(cudaMemset(H->status, 0, 4));
+  return s ? VLA_AE_ETIMEOUT : VLA_AE_OK;
+}
+
+int vla_ae_query(vla_ae_t H, int what, int arg, long long* value) {
+  if (!H || !value) return VLA_AE_EINVAL;
+  const vla_ae_dims& d = H->d;
+  switch (what) {
+    case VLA_AE_Q_KERNELS_PER_LOOP:
+      if (arg < 1) return VLA_AE_EINVAL;
+      *value = 1 + (long long)arg * (5LL * d.n_layers + 1);
+      return VLA_AE_OK;
+    case VLA_AE_Q_WEIGHT_BYTES: {
+      long long b = 0;
+      for (int id = 0; id < 4; ++id) b += (long long)H->op[id].wbytes;
+      if (H->fp8) b += (long long)H->layer_scales * 4;
+      *value = b * d.n_layers;
+      return VLA_AE_OK;
+    }
+    case VLA_AE_Q_KV_BYTES:
+      *value = 2LL * d.batch * d.n_layers * (long long)std::max(0, H->n_prefix) * d.n_kv_heads * d.head_dim * 2;
+      return VLA_AE_OK;
+    case VLA_AE_Q_DEVICE_BYTES:
+      *value = (long long)H->device_bytes;
+      return VLA_AE_OK;
+    case VLA_AE_Q_SPLITS:
+      *value = H->op[0].S | (H->op[1].S << 8) | (H->op[2].S << 16) | ((long long)H->op[3].S << 24);
+      return VLA_AE_OK;
+    default:
+      return VLA_AE_EINVAL;
+  }
+}
+
+int vla_ae_debug_layer(vla_ae_t H, int layer, int step, int steps, const float* h_in, float* h_out,
+                       const vla_ae_trace* trace) {
+  if (!H || !h_in || !h_out || layer < 0 || layer >= H->d.n_layers || steps < 1 || step < 0 || step >= steps)
+    return VLA_AE_EINVAL;
+  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+  StepTables* T = nullptr;
+  int rc = get_tables(H, steps, &T);
+  if (rc) return rc;
+  const size_t nh = (size_t)H->Ntok * H->d.hidden;
+  cudaStream_t st = H->cap;
+  CK(cudaMemcpyAsync(H->h, h_in, nh * 4, cudaMemcpyDeviceToDevice, st));
+  // partial sums of squares of h_in as a single part
+  row_sumsq_kernel<<<H->Ntok, 256, 0, st>>>(H->h, H->ss, H->d.hidden);
+  CK(cudaGetLastError());
+  CK(enqueue_layer(H, *T, step, layer, 1, st, trace));
+  CK(cudaMemcpyAsync(h_out, H->h, nh * 4, cudaMemcpyDeviceToDevice, st));
+  CK(cudaStreamSynchronize(st));
+  return VLA_AE_OK;
+}
+
+int vla_ae_debug_velocity(vla_ae_t H, int step, int steps, const float* x, float* v) {
+  if (!H || !x || !v || steps < 1 || step < 0 || step >= steps) return VLA_AE_EINVAL;
+  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+  StepTables* T = nullptr;
+  int rc = get_tables(H, steps, &T);
+  if (rc) return rc;
+  const vla_ae_dims& d = H->d;
+  cudaStream_t st = H->cap;
+  const size_t nx = (size_t)d.batch * d.n_action_tokens * d.action_dim;
+  CK(cudaMemcpyAsync(H->x, x, nx * 4, cudaMemcpyDeviceToDevice, st));
+  TailParams t0 = tail_common(H);
+  t0.do_in = 1;
+  CK(launch_tail(H, t0, st));
+  for (int l = 0; l < d.n_layers; ++l) CK(enqueue_layer(H, *T, step, l, l == 0 ? 1 : ss_parts_of(H, OP_D), st, nullptr));
+  TailParams t = tail_common(H);
+  t.ss_parts = ss_parts_of(H, OP_D);
+  t.shift_f = T->fmod + (size_t)step * 2 * d.hidden;
+  t.scale_f = t.shift_f + d.hidden;
+  t.dt = 0.f;
+  t.do_out = 1;
+  t.v_out = v;
+  CK(launch_tail(H, t, st));
+  CK(cudaStreamSynchronize(st));
+  return VLA_AE_OK;
+}
+
+int vla_ae_debug_weight(vla_ae_t H, int layer, int which, void* w_host, float* scales_host) {
+  if (!H || !w_host || layer < 0 || layer >= H->d.n_layers || which < 0 || which > 6) return VLA_AE_EINVAL;
+  const OpId id = which <= 2 ? OP_QKV : which == 3 ? OP_O : which <= 5 ? OP_GU : OP_D;
+  const OpPlan& p = H->op[id];
+  std::vector<uint8_t> blob(p.wbytes);
+  CK(cudaMemcpy(blob.data(), H->wpack + (size_t)layer * H->layer_wbytes + p.woff, p.wbytes, cudaMemcpyDeviceToHost));
+  std::vector<float> sc;
+  if (H->fp8) {
+    sc.resize((size_t)p.Mt * 128);
+    CK(cudaMemcpy(sc.data(), H->wscale + (size_t)layer * H->layer_scales + p.soff, sc.size() * 4,
+                  cudaMemcpyDeviceToHost));
+  }
+  const int K = p.K;
+  for (int pr = 0; pr < p.Mt * 128; ++pr) {
+    int mat, row;
+    packed_row_source(H, id, pr, &mat, &row);
+    if (mat != which) continue;
+    const int mt = pr / 128, r = pr % 128;
+    for (int k = 0; k < K; ++k) {
+      if (H->fp8) {
+        const size_t tile = (size_t)mt * p.KBt + k / 128;
+        const int kk = k % 128;
+        const size_t byte = tile * kTileBytes + sw128_chunk_byte(r, kk / 16) + (kk % 16);
+        reinterpret_cast<uint8_t*>(w_host)[(size_t)row * K + k] = blob[byte];
+      } else {
+        const size_t tile = (size_t)mt * p.KBt + k / 64;
+        const size_t elem = tile * (kTileBytes / 2) + sw128_elem_offset(r, k % 64);
+        reinterpret_cast<uint16_t*>(w_host)[(size_t)row * K + k] = reinterpret_cast<const uint16_t*>(blob.data())[elem];
+      }
+    }
+    if (H->fp8 && scales_host) scales_host[row] = sc[pr];
+  }
+  return VLA_AE_OK;
+}
+
+}  // extern "C"

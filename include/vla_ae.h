@@ -1,0 +1,160 @@
+/*
+ * vla_ae.h -- C ABI of the B200 (sm_100a) flow-matching action-expert denoise loop.
+ *
+ * The operation: the action expert of a vision-language-action model integrates
+ *     x_{k+1} = x_k + dt * v_theta(x_k, t_k, prefix KV),   t_k = 1 - k/N,  dt = -1/N,
+ * from Gaussian noise x_0 over N fixed Euler steps ("AI Infra如何优化VLA" (RimBot), section
+ * 整体方案: a 4-step x 36-layer DiT action head denoising from random noise; APXInf article,
+ * section "CUDA Graph、FP8 和 Rust": 10 flow steps, a 1-step variant and FP8 weights).
+ * v_theta is a DiT: per layer RMSNorm + adaLN time modulation, fused QKV projection with
+ * half-split RoPE, GQA attention of the action tokens over themselves and the cached VLM prefix
+ * K/V, o-projection, SwiGLU MLP and gated residual adds; an action out-projection closes it.
+ * ("跨XPU平台表征视觉-语言-动作模型" section 4.2: this stage is memory-bound.)
+ *
+ * Conventions for every entry point:
+ *   - returns VLA_AE_OK (0) or a negative VLA_AE_E* code; no exception crosses the ABI;
+ *   - calls taking a `stream` (a cudaStream_t, NULL = legacy default stream) only enqueue work
+ *     and return; results are ready when that stream reaches the enqueued work;
+ *   - a handle is not thread-safe; different handles are independent;
+ *   - the library allocates and owns all of its device memory; caller pointers are borrowed for
+ *     the duration of the call (or, for asynchronous calls, until the stream has consumed them).
+ * Data types: "bf16" = IEEE bfloat16 bit patterns (uint16), "fp32" = IEEE float.
+ */
+#ifndef VLA_AE_H
+#define VLA_AE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ status codes */
+#define VLA_AE_OK 0
+#define VLA_AE_EINVAL (-1)       /* bad argument: null pointer, dims out of range, n_prefix > max */
+#define VLA_AE_ENOMEM (-2)       /* device allocation failed */
+#define VLA_AE_ECUDA (-3)        /* a CUDA runtime call failed (no device, launch error, ...) */
+#define VLA_AE_ENOPREFIX (-4)    /* vla_ae_denoise before any vla_ae_set_prefix */
+#define VLA_AE_ETIMEOUT (-5)     /* a bounded device-side wait ran out (see vla_ae_status) */
+#define VLA_AE_EUNSUPPORTED (-6) /* valid dims this build does not implement (e.g. head_dim) */
+
+/* ------------------------------------------------------------------ configuration */
+typedef enum { VLA_AE_BF16 = 0, VLA_AE_FP8_E4M3 = 1 } vla_ae_wtype;
+
+/* Model and workload dimensions, fixed at create time.
+ * Requirements (else VLA_AE_EINVAL): every count >= 1 except has_state_token (0/1) and
+ * max_prefix (>= 0); hidden, inter % 8 == 0; head_dim in {64, 128, 256};
+ * n_q_heads % n_kv_heads == 0; t_emb_dim even; action_dim <= 64;
+ * batch * (n_action_tokens + has_state_token) <= 4096. */
+typedef struct {
+  int n_layers;         /* DiT layers L */
+  int hidden;           /* H */
+  int n_q_heads;        /* nq */
+  int n_kv_heads;       /* nkv (GQA: consecutive q heads share a kv head) */
+  int head_dim;         /* hd; q width nq*hd may differ from H */
+  int inter;            /* SwiGLU intermediate I */
+  int t_emb_dim;        /* sinusoidal time-embedding width Dt */
+  int action_dim;       /* A */
+  int n_action_tokens;  /* T (action chunk length) */
+  int has_state_token;  /* 1: one proprioceptive state token precedes the action tokens */
+  int max_prefix;       /* largest prefix length P accepted by vla_ae_set_prefix */
+  int batch;            /* B independent samples per call */
+  float rope_theta;     /* RoPE base (10000) */
+  float rms_eps;        /* RMSNorm epsilon (1e-6) */
+  int wtype;            /* vla_ae_wtype of the per-layer q/k/v/o/gate/up/down weights */
+} vla_ae_dims;
+
+/* Weights: bf16, matrices [out][in] row-major.  Per-layer entries are arrays of n_layers
+ * pointers.  adaLN per layer: w_ada [6H][Dt], b_ada [6H] in the order shift/scale/gate for the
+ * attention branch then for the MLP branch; final adaLN w_fada [2H][Dt], b_fada [2H] (shift,
+ * scale).  wq [nq*hd][H], wk/wv [nkv*hd][H], wo [H][nq*hd], wg/wu [I][H], wd [H][I];
+ * w_in/w_state [H][A], b_in/b_state [H], w_out [A][H], b_out [A]; w_state/b_state are ignored
+ * (may be NULL) without a state token.  on_device: 1 = all pointers are device memory,
+ * 0 = host memory; device per-layer matrices must be 16-byte aligned.  With wtype FP8 the library quantises q/k/v/o/gate/up/down itself (one fp32
+ * scale per output channel, scale = max|w|/448, codes = e4m3 round-to-nearest-even saturating
+ * of w/scale); everything else stays bf16.  The caller keeps ownership; the library copies. */
+typedef struct {
+  const void *w_in, *b_in, *w_state, *b_state;
+  const void *const *w_ada, *const *b_ada;
+  const void *const *wq, *const *wk, *const *wv, *const *wo;
+  const void *const *wg, *const *wu, *const *wd;
+  const void *w_fada, *b_fada, *w_out, *b_out;
+  int on_device;
+} vla_ae_weights;
+
+typedef struct vla_ae *vla_ae_t;
+
+/* Create a handle on the current CUDA device: validates dims, allocates every device buffer the
+ * loop needs, packs (and for FP8 quantises) the weights into the kernels' streaming layout.
+ * Synchronous.  Errors: EINVAL, EUNSUPPORTED, ENOMEM, ECUDA; *out is NULL on error. */
+int vla_ae_create(const vla_ae_dims *dims, const vla_ae_weights *weights, vla_ae_t *out);
+
+/* Set the cached VLM prefix for the next denoise calls (once per control cycle).
+ *   k, v   bf16 [B][L][n_prefix][nkv][hd], keys already rotated (RoPE applied by the VLM);
+ *   state  bf16 [B][A] proprioceptive state (required iff has_state_token, else ignored);
+ *   on_device: 1 = device pointers (copied device-to-device), 0 = host pointers.
+ * 0 <= n_prefix <= max_prefix.  Self tokens take positions n_prefix .. n_prefix+Ts-1.
+ * Asynchronous on `stream`.  Errors: EINVAL, ECUDA. */
+int vla_ae_set_prefix(vla_ae_t h, const void *k, const void *v, int n_prefix, const void *state,
+                      int on_device, void *stream);
+
+/* Run the N-step Euler loop.
+ *   noise  device bf16 [B][T][A], the initial x_0;
+ *   steps  N >= 1 (t_k = 1 - k/N, dt = -1/N);
+ *   out    device fp32 [B][T][A], receives x_N (caller-owned).
+ * The first call for a given `steps` builds that step count's adaLN table and captures the
+ * loop as one CUDA graph (do it before timing); later calls replay it.  Asynchronous on
+ * `stream`.  Errors: EINVAL, ENOPREFIX, ECUDA. */
+int vla_ae_denoise(vla_ae_t h, const void *noise, int steps, float *out, void *stream);
+
+/* Same as vla_ae_denoise with host buffers: noise_host bf16 [B][T][A] and out_host fp32
+ * [B][T][A] (pinned memory gives asynchronous copies).  Enqueues the host-to-device copy, the
+ * loop and the device-to-host copy on `stream`; out_host is valid after the stream syncs. */
+int vla_ae_denoise_host(vla_ae_t h, const void *noise_host, int steps, float *out_host, void *stream);
+
+/* Sticky device-side status: VLA_AE_OK, or VLA_AE_ETIMEOUT when a bounded wait inside a kernel
+ * ran out (the results of that call are invalid).  Synchronises the device.  Clears the flag. */
+int vla_ae_status(vla_ae_t h);
+
+/* Static text for a status code. */
+const char *vla_ae_strerror(int code);
+
+/* Release every resource of the handle (synchronises the device).  NULL is a no-op. */
+void vla_ae_destroy(vla_ae_t h);
+
+/* ------------------------------------------------------------------ introspection */
+#define VLA_AE_Q_KERNELS_PER_LOOP 1   /* kernel launches per denoise loop of `arg` steps */
+#define VLA_AE_Q_WEIGHT_BYTES 2       /* bytes of streamed linear weights (+fp8 scales) per step */
+#define VLA_AE_Q_KV_BYTES 3           /* bytes of prefix K+V read per step (whole batch) */
+#define VLA_AE_Q_DEVICE_BYTES 4       /* device memory held by the handle */
+#define VLA_AE_Q_SPLITS 5             /* packed split-K of the four GEMMs: qkv | o<<8 | gu<<16 | d<<24 */
+/* Query a property of the handle into *value.  Errors: EINVAL. */
+int vla_ae_query(vla_ae_t h, int what, int arg, long long *value);
+
+/* ------------------------------------------------------------------ test hooks
+ * Teacher-forced execution of one DiT layer (per-layer parity): h_in and h_out are device fp32
+ * [B*Ts][H] (row b*Ts + j is token j of sample b; j = 0 is the state token when present);
+ * the layer uses the adaLN table of step `step` out of `steps` and the current prefix.
+ * Any non-NULL trace pointer (device fp32) receives an intermediate, row per token:
+ *   q [B*Ts][nq*hd] and k, v [B*Ts][nkv*hd] after RoPE (v unrotated), o [B*Ts][nq*hd] attention
+ *   output, h_attn [B*Ts][H] after the attention residual, m [B*Ts][I] SwiGLU output.
+ * Synchronous.  Errors: EINVAL, ENOPREFIX, ECUDA. */
+typedef struct {
+  float *q, *k, *v, *o, *h_attn, *m;
+} vla_ae_trace;
+int vla_ae_debug_layer(vla_ae_t h, int layer, int step, int steps, const float *h_in, float *h_out,
+                       const vla_ae_trace *trace);
+
+/* v_theta(x, t_step) for device fp32 x [B][T][A] into device fp32 v [B][T][A].  Synchronous. */
+int vla_ae_debug_velocity(vla_ae_t h, int step, int steps, const float *x, float *v);
+
+/* Read back one packed per-layer weight in [out][in] order (which: 0 q, 1 k, 2 v, 3 o, 4 gate,
+ * 5 up, 6 down) into host memory: bf16 weights as uint16 bits, FP8 weights as e4m3 codes
+ * (uint8) plus fp32 scales [out] (scales may be NULL for bf16).  Synchronous. */
+int vla_ae_debug_weight(vla_ae_t h, int layer, int which, void *w_host, float *scales_host);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VLA_AE_H */

@@ -39,7 +39,7 @@ import numpy as np
 __all__ = [
     "Dims", "CONFIGS", "config", "f32_to_bf16_bits", "bf16_bits_to_f32",
     "generate_weights", "generate_sample", "generate_inputs", "WEIGHT_ORDER",
-    "LAYER_WEIGHT_ORDER", "weight_shapes",
+    "LAYER_WEIGHT_ORDER", "weight_shapes", "abi_dims", "BATCH_SWEEP",
 ]
 
 
@@ -200,3 +200,12 @@ def generate_inputs(d: Dims, seed: int = 0, n_prefix: int | None = None) -> Dict
     samples = [generate_sample(d, b, seed, n_prefix) for b in range(d.batch)]
     out = {key: np.stack([s[key] for s in samples]) for key in samples[0]}
     return out
+
+
+def abi_dims(d: Dims, max_prefix: int | None = None) -> Dict[str, object]:
+    """The ``vla_ae_dims`` fields for a workload (field renaming only)."""
+    return dict(n_layers=d.n_layers, hidden=d.hidden, n_q_heads=d.n_q_heads, n_kv_heads=d.n_kv_heads,
+                head_dim=d.head_dim, inter=d.inter, t_emb_dim=d.t_emb_dim, action_dim=d.action_dim,
+                n_action_tokens=d.n_action_tokens, has_state_token=d.has_state_token,
+                max_prefix=d.n_prefix if max_prefix is None else max_prefix, batch=d.batch,
+                rope_theta=d.rope_theta, rms_eps=d.rms_eps, wtype=0 if d.wtype == "bf16" else 1)
