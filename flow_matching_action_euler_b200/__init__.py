@@ -17,12 +17,12 @@ __all__ = [
     "lib", "VlaAeDims", "VlaAeWeights", "VlaAeTrace", "VlaAeError", "ActionExpert",
     "vla_ae_create", "vla_ae_set_prefix", "vla_ae_denoise", "vla_ae_denoise_host", "vla_ae_status",
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
-    "vla_ae_debug_weight", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
-    "Q_DEVICE_BYTES", "Q_SPLITS",
+    "vla_ae_debug_weight", "vla_ae_bench_op", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
+    "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES",
 ]
 
 BF16, FP8_E4M3 = 0, 1
-Q_KERNELS_PER_LOOP, Q_WEIGHT_BYTES, Q_KV_BYTES, Q_DEVICE_BYTES, Q_SPLITS = 1, 2, 3, 4, 5
+Q_KERNELS_PER_LOOP, Q_WEIGHT_BYTES, Q_KV_BYTES, Q_DEVICE_BYTES, Q_SPLITS, Q_OP_BYTES = 1, 2, 3, 4, 5, 6
 OK, EINVAL, ENOMEM, ECUDA, ENOPREFIX, ETIMEOUT, EUNSUPPORTED = 0, -1, -2, -3, -4, -5, -6
 
 if not os.path.exists(LIB_PATH):
@@ -76,6 +76,7 @@ vla_ae_debug_layer = _sig("vla_ae_debug_layer", ctypes.c_int, _H, ctypes.c_int, 
                           ctypes.POINTER(VlaAeTrace))
 vla_ae_debug_velocity = _sig("vla_ae_debug_velocity", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_debug_weight = _sig("vla_ae_debug_weight", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, _P, _P)
+vla_ae_bench_op = _sig("vla_ae_bench_op", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P)
 
 
 class VlaAeError(RuntimeError):
@@ -173,6 +174,9 @@ class ActionExpert:
 
     def debug_weight(self, layer: int, which: int, w_host, scales_host=None):
         _check(vla_ae_debug_weight(self.handle, layer, which, _ptr(w_host), _ptr(scales_host)), "vla_ae_debug_weight")
+
+    def bench_op(self, op: int, count: int, steps: int, stream=None):
+        _check(vla_ae_bench_op(self.handle, op, count, steps, _stream_ptr(stream)), "vla_ae_bench_op")
 
     def close(self):
         if getattr(self, "handle", None):

@@ -68,7 +68,7 @@ struct GemmParams {
   int nq, nkv, hd, Ts, P, Lpad;
   unsigned* status;
   // ---- shared-memory layout (bytes from the 1024-aligned base)
-  int off_b, off_conv, off_bar, smem_bytes;
+  int off_b, off_conv, off_bar, off_misc, kmax, smem_bytes;
 };
 
 __device__ __forceinline__ void math_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -99,7 +99,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
   uint64_t* cfull = done + 1;                             // [kConvStages]
   uint64_t* cempty = cfull + kConvStages;                 // [kConvStages]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cempty + kConvStages);
-  float* rstd = reinterpret_cast<float*>(tmem_slot + 4);  // [NT]
+  float* s_shift = reinterpret_cast<float*>(smem + p.off_misc);   // [kmax] modulation slice of this CTA
+  float* s_scale = s_shift + p.kmax;                              // [kmax]
+  float* rpart = s_scale + p.kmax;                                // [256] partial sums of squares
+  float* rstd = rpart + kMathThreads;                             // [NT]
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.stages; ++i) {
@@ -234,45 +237,98 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
       const int pre = min(nkt, kConvStages);
       for (; conv_done < pre && ok; ++conv_done) ok = convert_one(conv_done);
     }
+    const int nkb = kb1 - kb0;
+    if (BMODE == B_NORM) {
+      // the modulation vectors are input-independent: stage this CTA's slice before waiting
+      for (int i = mtid; i < nkb * 64; i += kMathThreads) {
+        const int k = kb0 * 64 + i;
+        s_shift[i] = k < p.K ? __ldg(p.shift + k) : 0.f;
+        s_scale[i] = k < p.K ? __ldg(p.scale + k) : 0.f;
+      }
+    }
     pdl_wait();
     if (BMODE == B_NORM) {
-      // u = rms(h) * (1 + scale) + shift, bf16, written straight into the swizzled B tiles
-      if (mtid < NT) {
-        const int t = nt * NT + mtid;
+      // rstd per token row from the producers' partial sums of squares: G threads per row each
+      // take every G-th part, then the G partials are added in a fixed order (deterministic)
+      const int G = NT >= kMathThreads ? 1 : kMathThreads / NT;
+      {
+        const int row = mtid / G, g = mtid % G;
+        const int t = nt * NT + row;
         float acc = 0.f;
-        if (t < p.Ntok)
-          for (int q = 0; q < p.ss_parts; ++q) acc += p.ss[(size_t)q * p.Ntok + t];
-        rstd[mtid] = rsqrtf(acc / (float)p.K + p.eps);
+        if (row < NT && t < p.Ntok) {
+          int q = g;
+          for (; q + 3 * G < p.ss_parts; q += 4 * G) {
+            const float a0 = __ldcg(p.ss + (size_t)q * p.Ntok + t);
+            const float a1 = __ldcg(p.ss + (size_t)(q + G) * p.Ntok + t);
+            const float a2 = __ldcg(p.ss + (size_t)(q + 2 * G) * p.Ntok + t);
+            const float a3 = __ldcg(p.ss + (size_t)(q + 3 * G) * p.Ntok + t);
+            acc += a0;
+            acc += a1;
+            acc += a2;
+            acc += a3;
+          }
+          for (; q < p.ss_parts; q += G) acc += __ldcg(p.ss + (size_t)q * p.Ntok + t);
+        }
+        rpart[mtid] = acc;
       }
       math_bar();
-      const int nkb = kb1 - kb0;
-      const int nchunks = NT * nkb * 8;
-      for (int e = mtid; e < nchunks; e += kMathThreads) {
-        const int ch = e & 7, rest = e >> 3;
-        const int row = rest % NT, lk = rest / NT;
-        const int t = nt * NT + row;
-        const int k = (kb0 + lk) * 64 + ch * 8;
-        uint4 packed = make_uint4(0, 0, 0, 0);
-        if (t < p.Ntok && k < p.K) {
-          const float4* hp = reinterpret_cast<const float4*>(p.h + (size_t)t * p.K + k);
-          const float4* sh = reinterpret_cast<const float4*>(p.shift + k);
-          const float4* sc = reinterpret_cast<const float4*>(p.scale + k);
-          const float rs = rstd[row];
-          float v[8];
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const float4 a = hp[hh], b = sh[hh], c = sc[hh];
-            v[4 * hh + 0] = a.x * rs * (1.f + c.x) + b.x;
-            v[4 * hh + 1] = a.y * rs * (1.f + c.y) + b.y;
-            v[4 * hh + 2] = a.z * rs * (1.f + c.z) + b.z;
-            v[4 * hh + 3] = a.w * rs * (1.f + c.w) + b.w;
-          }
-          __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[4], v[5]), b3 = __floats2bfloat162_rn(v[6], v[7]);
-          packed = make_uint4(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1),
-                              *reinterpret_cast<uint32_t*>(&b2), *reinterpret_cast<uint32_t*>(&b3));
+      for (int row = mtid; row < NT; row += kMathThreads) {
+        float acc = 0.f;
+        if (NT >= kMathThreads) {
+          acc = rpart[row];   // G == 1: one thread per row already summed everything
+        } else {
+          for (int g = 0; g < G; ++g) acc += rpart[row * G + g];
         }
-        *reinterpret_cast<uint4*>(sB + (size_t)lk * NT * 128 + sw128_chunk_byte(row, ch)) = packed;
+        rstd[row] = rsqrtf(acc / (float)p.K + p.eps);
+      }
+      math_bar();
+      // u = rms(h) * (1 + scale) + shift -> bf16, written straight into the swizzled B tiles;
+      // loads are issued in batches of 4 chunks so their latencies overlap
+      const int nchunks = NT * nkb * 8;
+      for (int e0 = mtid; e0 < nchunks; e0 += 4 * kMathThreads) {
+        float4 hv[4][2];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u * kMathThreads;
+          const int ch = e & 7, rest = e >> 3;
+          const int row = rest % NT, lk = rest / NT;
+          const int t = nt * NT + row;
+          const int k = (kb0 + lk) * 64 + ch * 8;
+          if (e < nchunks && t < p.Ntok && k < p.K) {
+            const float4* hp = reinterpret_cast<const float4*>(p.h + (size_t)t * p.K + k);
+            hv[u][0] = __ldcg(hp);
+            hv[u][1] = __ldcg(hp + 1);
+          } else {
+            hv[u][0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            hv[u][1] = hv[u][0];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = e0 + u * kMathThreads;
+          if (e >= nchunks) break;
+          const int ch = e & 7, rest = e >> 3;
+          const int row = rest % NT, lk = rest / NT;
+          const int t = nt * NT + row;
+          const int kl = lk * 64 + ch * 8;
+          const int k = kb0 * 64 + kl;
+          uint4 packed = make_uint4(0, 0, 0, 0);
+          if (t < p.Ntok && k < p.K) {
+            const float rs = rstd[row];
+            const float hvals[8] = {hv[u][0].x, hv[u][0].y, hv[u][0].z, hv[u][0].w,
+                                    hv[u][1].x, hv[u][1].y, hv[u][1].z, hv[u][1].w};
+            uint32_t w4[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float v0 = hvals[2 * q] * rs * (1.f + s_scale[kl + 2 * q]) + s_shift[kl + 2 * q];
+              const float v1 = hvals[2 * q + 1] * rs * (1.f + s_scale[kl + 2 * q + 1]) + s_shift[kl + 2 * q + 1];
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+              w4[q] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            packed = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+          *reinterpret_cast<uint4*>(sB + (size_t)lk * NT * 128 + sw128_chunk_byte(row, ch)) = packed;
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(bfull);
@@ -314,11 +370,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
       float y0 = 0.f, y1 = 0.f;
       const uint32_t off = (uint32_t)(col * 128 + 2 * pr) * 4u;
       if (S > 1) {
-        for (int s = 0; s < S; ++s) {   // fixed order: deterministic
-          const uint32_t a = mapa_shared(red_local + off, (uint32_t)s);
-          y0 += ld_dsmem_f32(a);
-          y1 += ld_dsmem_f32(a + 4);
-        }
+        // all S remote loads in flight first, then the sum in rank order (deterministic)
+        float2 part[16];
+#pragma unroll
+        for (int s = 0; s < 16; ++s)
+          if (s < S) part[s] = ld_dsmem_f32x2(mapa_shared(red_local + off, (uint32_t)s));
+#pragma unroll
+        for (int s = 0; s < 16; ++s)
+          if (s < S) {
+            y0 += part[s].x;
+            y1 += part[s].y;
+          }
       } else {
         y0 = red[col * 128 + 2 * pr];
         y1 = red[col * 128 + 2 * pr + 1];
@@ -331,11 +393,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
       if (EPI == EPI_RESID) {
         float hsq = 0.f;
         if (valid) {
-          float* hp = p.h_out + (size_t)t * p.O + o0;
-          const float hn0 = hp[0] + p.gate[o0] * y0;
-          const float hn1 = hp[1] + p.gate[o0 + 1] * y1;
-          hp[0] = hn0;
-          hp[1] = hn1;
+          float2* hp = reinterpret_cast<float2*>(p.h_out + (size_t)t * p.O + o0);
+          const float2 ho = __ldcg(hp);
+          const float hn0 = ho.x + __ldg(p.gate + o0) * y0;
+          const float hn1 = ho.y + __ldg(p.gate + o0 + 1) * y1;
+          __stcg(hp, make_float2(hn0, hn1));
           hsq = hn0 * hn0 + hn1 * hn1;
         }
         sq[col * npairs + (e % npairs)] = hsq;

@@ -39,8 +39,9 @@ struct TailParams {
 };
 
 __global__ void __launch_bounds__(kTailThreads) tail_kernel(const __grid_constant__ TailParams p) {
-  __shared__ float red[kTailThreads / 32][kMaxAction];
+  __shared__ float vsh[kMaxAction];
   __shared__ float xs[kMaxAction];
+  __shared__ float red[kTailThreads / 32];
   __shared__ float rs_sh;
   const int t = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = t / p.Ts, j = t % p.Ts;
@@ -50,80 +51,64 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const __grid_constan
   pdl_trigger();
   pdl_wait();
   float* hrow = p.h + (size_t)t * H;
-  if (!is_state) {
-    float* xrow = p.x + ((size_t)b * p.T + a_row) * A;
-    if (p.init_from_noise) {
-      if (tid < A) xrow[tid] = __bfloat162float(p.noise[((size_t)b * p.T + a_row) * A + tid]);
-      __syncthreads();
-    }
-    if (p.do_out) {
-      if (tid == 0) {
-        float acc = 0.f;
-        for (int q = 0; q < p.ss_parts; ++q) acc += p.ss[(size_t)q * p.Ntok + t];
-        rs_sh = rsqrtf(acc / (float)H + p.eps);
-      }
-      __syncthreads();
-      const float rs = rs_sh;
-      float part[kMaxAction];
-      for (int a = 0; a < A; ++a) part[a] = 0.f;
-      for (int k = tid; k < H; k += kTailThreads) {
-        const float u = hrow[k] * rs * (1.f + p.scale_f[k]) + p.shift_f[k];
-        for (int a = 0; a < A; ++a) part[a] = fmaf(__bfloat162float(p.w_out[(size_t)a * H + k]), u, part[a]);
-      }
-      // fixed-order block reduction: warp shuffle tree, then warps in order
-      for (int a = 0; a < A; ++a) {
-        float v = part[a];
+  float* xrow = is_state ? nullptr : p.x + ((size_t)b * p.T + a_row) * A;
+  if (!is_state && p.init_from_noise && tid < A)
+    xrow[tid] = __bfloat162float(p.noise[((size_t)b * p.T + a_row) * A + tid]);
+  if (!is_state && p.do_out) {
+    if (warp == 0) {   // rstd from the down GEMM's partial sums of squares (fixed order)
+      float acc = 0.f;
+      for (int q = lane; q < p.ss_parts; q += 32) acc += __ldcg(p.ss + (size_t)q * p.Ntok + t);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[warp][a] = v;
-      }
-      __syncthreads();
-      if (tid < A) {
-        float v = __bfloat162float(p.b_out[tid]);
-        for (int w = 0; w < kTailThreads / 32; ++w) v += red[w][tid];
-        if (p.v_out) p.v_out[((size_t)b * p.T + a_row) * A + tid] = v;
-        const float xn = xrow[tid] + p.dt * v;
-        xrow[tid] = xn;
-        if (p.out) p.out[((size_t)b * p.T + a_row) * A + tid] = xn;
-      }
-      __syncthreads();
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) rs_sh = rsqrtf(acc / (float)H + p.eps);
     }
-    if (p.do_in) {
-      if (tid < A) xs[tid] = xrow[tid];
-      __syncthreads();
-      float sq = 0.f;
-      for (int o = tid; o < H; o += kTailThreads) {
-        float v = __bfloat162float(p.b_in[o]);
-        for (int a = 0; a < A; ++a) v = fmaf(__bfloat162float(p.w_in[(size_t)o * A + a]), xs[a], v);
-        hrow[o] = v;
-        sq = fmaf(v, v, sq);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (lane == 0) red[warp][0] = sq;
-      __syncthreads();
-      if (tid == 0) {
-        float s = 0.f;
-        for (int w = 0; w < kTailThreads / 32; ++w) s += red[w][0];
-        p.ss_out[t] = s;
-      }
-    }
-  } else if (p.do_in) {
-    float sq = 0.f;
-    for (int o = tid; o < H; o += kTailThreads) {
-      const float v = p.h_state0[(size_t)b * H + o];
-      hrow[o] = v;
-      sq = fmaf(v, v, sq);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (lane == 0) red[warp][0] = sq;
     __syncthreads();
-    if (tid == 0) {
-      float s = 0.f;
-      for (int w = 0; w < kTailThreads / 32; ++w) s += red[w][0];
-      p.ss_out[t] = s;
+    const float rs = rs_sh;
+    // v[a] = W_out[a] . (rms(h) (1 + sc_f) + sh_f) + b_out[a]: one warp per output, lanes over k
+    for (int a = warp; a < A; a += kTailThreads / 32) {
+      float acc = 0.f;
+      for (int k = lane; k < H; k += 32) {
+        const float u = __ldcg(hrow + k) * rs * (1.f + __ldg(p.scale_f + k)) + __ldg(p.shift_f + k);
+        acc = fmaf(__bfloat162float(p.w_out[(size_t)a * H + k]), u, acc);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) vsh[a] = acc + __bfloat162float(p.b_out[a]);
     }
+    __syncthreads();
+    if (tid < A) {
+      const float v = vsh[tid];
+      if (p.v_out) p.v_out[((size_t)b * p.T + a_row) * A + tid] = v;
+      const float xn = xrow[tid] + p.dt * v;
+      xrow[tid] = xn;
+      if (p.out) p.out[((size_t)b * p.T + a_row) * A + tid] = xn;
+    }
+  }
+  if (!p.do_in) return;
+  __syncthreads();
+  if (!is_state && tid < A) xs[tid] = xrow[tid];
+  __syncthreads();
+  // next step's self-token row: W_in x + b_in (action rows) or the cached state projection
+  float sq = 0.f;
+  for (int o = tid; o < H; o += kTailThreads) {
+    float v;
+    if (is_state) {
+      v = p.h_state0[(size_t)b * H + o];
+    } else {
+      v = __bfloat162float(p.b_in[o]);
+      for (int a = 0; a < A; ++a) v = fmaf(__bfloat162float(p.w_in[(size_t)o * A + a]), xs[a], v);
+    }
+    hrow[o] = v;
+    sq = fmaf(v, v, sq);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if (lane == 0) red[warp] = sq;
+  __syncthreads();
+  if (tid == 0) {
+    float s = 0.f;
+    for (int w = 0; w < kTailThreads / 32; ++w) s += red[w];
+    p.ss_out[t] = s;
   }
 }
 

@@ -52,7 +52,7 @@ struct OpPlan {
   size_t wbytes = 0;        // packed tile bytes of one layer
   size_t woff = 0;          // offset inside a layer's packed block
   size_t soff = 0;          // offset of the op's scales inside a layer's scale block (floats)
-  int off_b = 0, off_conv = 0, off_bar = 0, smem = 0;
+  int off_b = 0, off_conv = 0, off_bar = 0, off_misc = 0, kmax = 0, smem = 0;
 };
 
 struct StepTables {
@@ -169,8 +169,11 @@ void gemm_layout(OpPlan& p, int NT, bool fp8) {
   p.off_b = (int)a_region;
   p.off_conv = (int)(a_region + b_region);
   p.off_bar = (int)(a_region + b_region + conv);
-  const size_t bar_bytes = 8 * (2 * p.stages + 2 + 2 * kConvStages) + 16 + 4 * NT;
-  p.smem = (int)(p.off_bar + align_up(bar_bytes, 16) + 1024);   // + alignment slack
+  const size_t bar_bytes = 8 * (2 * p.stages + 2 + 2 * kConvStages) + 16;
+  p.off_misc = (int)(p.off_bar + align_up(bar_bytes, 16));
+  p.kmax = nkb_max * 64;
+  const size_t misc = 4 * (2 * (size_t)p.kmax + kMathThreads + NT);
+  p.smem = (int)(p.off_misc + align_up(misc, 16) + 1024);   // + alignment slack
 }
 
 int plan_gemm(vla_ae* H, OpPlan& p, OpId id, int O, int K) {
@@ -289,21 +292,24 @@ int plan_attention(vla_ae* H, int P) {
   std::vector<int> cands;
   for (int c = S; c >= 1; --c) cands.push_back(c);
   for (int c = S + 1; c <= std::min(16, L); ++c) cands.push_back(c);
-  for (int S : cands) {
-    const int cmax = ceil_div(L, S);
+  for (int S0 : cands) {
+    const int cs = (int)align_up((size_t)ceil_div(L, S0), 16);   // keys per chunk, multiple of 16
+    const int S = ceil_div(L, cs);
     const int Ts = H->Ts;
-    size_t off = (size_t)Ts * hd * 4;
+    size_t off = (size_t)Ts * (hd + 8) * 2;
     AttnParams a{};
+    off = align_up(off, 16);
     a.off_k = (int)off;
-    off = align_up(off + (size_t)cmax * (hd + 2) * 2, 16);
+    off = align_up(off + (size_t)cs * (hd + 8) * 2, 16);
     a.off_v = (int)off;
-    off = align_up(off + (size_t)hd * (cmax + 2) * 2, 16);
+    off = align_up(off + (size_t)hd * (cs + 8) * 2, 16);
     a.off_s = (int)off;
-    off = align_up(off + (size_t)Ts * cmax * 4, 16);
+    off = align_up(off + (size_t)Ts * cs * 4, 16);
     a.off_o = (int)off;
     off = align_up(off + (size_t)Ts * hd * 4, 16);
     a.off_ml = (int)off;
     off += (size_t)(2 + 16) * Ts * 4;
+    a.cs = cs;
     a.smem_bytes = (int)off;
     if (off > (size_t)kMaxDynSmem) continue;
     if (S > 1) {
@@ -326,7 +332,7 @@ int plan_attention(vla_ae* H, int P) {
       if (ncl < 1) continue;
     }
     H->attn_S = S;
-    H->attn_cmax = cmax;
+    H->attn_cmax = cs;
     H->attn_smem = (int)off;
     H->attn_proto = a;
     return VLA_AE_OK;
@@ -364,6 +370,8 @@ GemmParams gemm_common(const vla_ae* H, OpId id, int layer) {
   g.off_b = p.off_b;
   g.off_conv = p.off_conv;
   g.off_bar = p.off_bar;
+  g.off_misc = p.off_misc;
+  g.kmax = p.kmax;
   g.smem_bytes = p.smem;
   return g;
 }
@@ -375,92 +383,105 @@ cudaError_t launch_gemm(const vla_ae* H, OpId id, const GemmParams& g, cudaStrea
 
 int ss_parts_of(const vla_ae* H, OpId id) { return H->op[id].Mt * H->op[id].S; }
 
-// The five kernels of one DiT layer.  `ss_in_parts`: partial sums of squares feeding the first norm.
-cudaError_t enqueue_layer(vla_ae* H, const StepTables& T, int step, int layer, int ss_in_parts, cudaStream_t st,
-                          const vla_ae_trace* trace) {
+// Kernels of one DiT layer, in loop order.
+enum LayerOp { LOP_QKV = 0, LOP_ATTN = 1, LOP_O = 2, LOP_GU = 3, LOP_D = 4 };
+
+// One kernel of layer `layer` at step `step`.  `ss_in_parts`: partial sums of squares feeding
+// the QKV kernel's RMSNorm (1 after the in-projection, Mt*S of the down GEMM otherwise).
+cudaError_t enqueue_op(vla_ae* H, const StepTables& T, int step, int layer, int op, int ss_in_parts,
+                       cudaStream_t st) {
   const vla_ae_dims& d = H->d;
   const LayerPtrs m = layer_mod(H, T, step, layer);
   const size_t cache = (size_t)layer * d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+  switch (op) {
+    case LOP_QKV: {  // RMSNorm + modulate -> QKV -> RoPE -> q, K/V caches
+      GemmParams g = gemm_common(H, OP_QKV, layer);
+      g.h = H->h;
+      g.ss = H->ss;
+      g.ss_parts = ss_in_parts;
+      g.shift = m.shift_a;
+      g.scale = m.scale_a;
+      g.q_out = H->q;
+      g.kc = H->kc + cache;
+      g.vct = H->vct + cache;
+      g.rope = H->rope;
+      g.nq = d.n_q_heads;
+      g.nkv = d.n_kv_heads;
+      g.hd = d.head_dim;
+      g.Ts = H->Ts;
+      g.P = H->n_prefix;
+      g.Lpad = H->Lpad;
+      return launch_gemm(H, OP_QKV, g, st);
+    }
+    case LOP_ATTN: {  // attention over prefix + self
+      AttnParams a = H->attn_proto;
+      a.q = H->q;
+      a.kc = H->kc + cache;
+      a.vct = H->vct + cache;
+      a.o_tiles = H->act_o;
+      a.nq = d.n_q_heads;
+      a.nkv = d.n_kv_heads;
+      a.hd = d.head_dim;
+      a.Ts = H->Ts;
+      a.P = H->n_prefix;
+      a.Lpad = H->Lpad;
+      a.Ntok = H->Ntok;
+      a.NT = H->NT;
+      a.KBo = H->op[OP_O].KB;
+      a.S = H->attn_S;
+      a.cs = H->attn_cmax;
+      a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
+      return launch(attn_kernel_for(d.head_dim), dim3(H->attn_S, d.n_q_heads, d.batch), dim3(kAttnThreads),
+                    H->attn_smem, st, H->attn_S, true, a);
+    }
+    case LOP_O: {  // o-projection + gated residual
+      GemmParams g = gemm_common(H, OP_O, layer);
+      g.act = H->act_o;
+      g.h_out = H->h;
+      g.gate = m.gate_a;
+      g.ss_out = H->ss;
+      return launch_gemm(H, OP_O, g, st);
+    }
+    case LOP_GU: {  // RMSNorm + modulate -> gate/up -> SwiGLU
+      GemmParams g = gemm_common(H, OP_GU, layer);
+      g.h = H->h;
+      g.ss = H->ss;
+      g.ss_parts = ss_parts_of(H, OP_O);
+      g.shift = m.shift_m;
+      g.scale = m.scale_m;
+      g.m_out = H->act_m;
+      g.KBm = H->op[OP_D].KB;
+      return launch_gemm(H, OP_GU, g, st);
+    }
+    default: {  // down-projection + gated residual
+      GemmParams g = gemm_common(H, OP_D, layer);
+      g.act = H->act_m;
+      g.h_out = H->h;
+      g.gate = m.gate_m;
+      g.ss_out = H->ss;
+      return launch_gemm(H, OP_D, g, st);
+    }
+  }
+}
+
+cudaError_t enqueue_layer(vla_ae* H, const StepTables& T, int step, int layer, int ss_in_parts, cudaStream_t st,
+                          const vla_ae_trace* trace) {
+  const vla_ae_dims& d = H->d;
+  const size_t cache = (size_t)layer * d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
   cudaError_t e;
-  {  // RMSNorm + modulate -> QKV -> RoPE -> q, K/V caches
-    GemmParams g = gemm_common(H, OP_QKV, layer);
-    g.h = H->h;
-    g.ss = H->ss;
-    g.ss_parts = ss_in_parts;
-    g.shift = m.shift_a;
-    g.scale = m.scale_a;
-    g.q_out = H->q;
-    g.kc = H->kc + cache;
-    g.vct = H->vct + cache;
-    g.rope = H->rope;
-    g.nq = d.n_q_heads;
-    g.nkv = d.n_kv_heads;
-    g.hd = d.head_dim;
-    g.Ts = H->Ts;
-    g.P = H->n_prefix;
-    g.Lpad = H->Lpad;
-    if ((e = launch_gemm(H, OP_QKV, g, st)) != cudaSuccess) return e;
-  }
-  if (trace && (trace->q || trace->k || trace->v)) {
-    if (trace->q) bf16_to_f32_kernel<<<64, 256, 0, st>>>(H->q, trace->q, (size_t)H->Ntok * H->qd);
-    if (trace->k && trace->v)
-      self_kv_kernel<<<64, 256, 0, st>>>(H->kc + cache, H->vct + cache, trace->k, trace->v, d.batch, H->Ts,
-                                         d.n_kv_heads, d.head_dim, H->n_prefix, H->Lpad);
-  }
-  {  // attention over prefix + self
-    AttnParams a = H->attn_proto;
-    a.q = H->q;
-    a.kc = H->kc + cache;
-    a.vct = H->vct + cache;
-    a.o_tiles = H->act_o;
-    a.nq = d.n_q_heads;
-    a.nkv = d.n_kv_heads;
-    a.hd = d.head_dim;
-    a.Ts = H->Ts;
-    a.P = H->n_prefix;
-    a.Lpad = H->Lpad;
-    a.Ntok = H->Ntok;
-    a.NT = H->NT;
-    a.KBo = H->op[OP_O].KB;
-    a.S = H->attn_S;
-    a.cmax = H->attn_cmax;
-    a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
-    if ((e = launch(attn_kernel_for(d.head_dim), dim3(H->attn_S, d.n_q_heads, d.batch), dim3(kAttnThreads),
-                    H->attn_smem, st, H->attn_S, true, a)) != cudaSuccess)
-      return e;
-  }
+  if ((e = enqueue_op(H, T, step, layer, LOP_QKV, ss_in_parts, st)) != cudaSuccess) return e;
+  if (trace && trace->q) bf16_to_f32_kernel<<<64, 256, 0, st>>>(H->q, trace->q, (size_t)H->Ntok * H->qd);
+  if (trace && trace->k && trace->v)
+    self_kv_kernel<<<64, 256, 0, st>>>(H->kc + cache, H->vct + cache, trace->k, trace->v, d.batch, H->Ts,
+                                       d.n_kv_heads, d.head_dim, H->n_prefix, H->Lpad);
+  if ((e = enqueue_op(H, T, step, layer, LOP_ATTN, 0, st)) != cudaSuccess) return e;
   if (trace && trace->o) untile_kernel<<<64, 256, 0, st>>>(H->act_o, trace->o, H->Ntok, H->qd, H->NT, H->op[OP_O].KB);
-  {  // o-projection + gated residual
-    GemmParams g = gemm_common(H, OP_O, layer);
-    g.act = H->act_o;
-    g.h_out = H->h;
-    g.gate = m.gate_a;
-    g.ss_out = H->ss;
-    if ((e = launch_gemm(H, OP_O, g, st)) != cudaSuccess) return e;
-  }
+  if ((e = enqueue_op(H, T, step, layer, LOP_O, 0, st)) != cudaSuccess) return e;
   if (trace && trace->h_attn)
     cudaMemcpyAsync(trace->h_attn, H->h, (size_t)H->Ntok * d.hidden * 4, cudaMemcpyDeviceToDevice, st);
-  {  // RMSNorm + modulate -> gate/up -> SwiGLU
-    GemmParams g = gemm_common(H, OP_GU, layer);
-    g.h = H->h;
-    g.ss = H->ss;
-    g.ss_parts = ss_parts_of(H, OP_O);
-    g.shift = m.shift_m;
-    g.scale = m.scale_m;
-    g.m_out = H->act_m;
-    g.KBm = H->op[OP_D].KB;
-    if ((e = launch_gemm(H, OP_GU, g, st)) != cudaSuccess) return e;
-  }
+  if ((e = enqueue_op(H, T, step, layer, LOP_GU, 0, st)) != cudaSuccess) return e;
   if (trace && trace->m) untile_kernel<<<64, 256, 0, st>>>(H->act_m, trace->m, H->Ntok, d.inter, H->NT, H->op[OP_D].KB);
-  {  // down-projection + gated residual
-    GemmParams g = gemm_common(H, OP_D, layer);
-    g.act = H->act_m;
-    g.h_out = H->h;
-    g.gate = m.gate_m;
-    g.ss_out = H->ss;
-    if ((e = launch_gemm(H, OP_D, g, st)) != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  return enqueue_op(H, T, step, layer, LOP_D, 0, st);
 }
 
 TailParams tail_common(const vla_ae* H) {
@@ -848,12 +869,36 @@ int vla_ae_query(vla_ae_t H, int what, int arg, long long* value) {
     case VLA_AE_Q_DEVICE_BYTES:
       *value = (long long)H->device_bytes;
       return VLA_AE_OK;
+    case VLA_AE_Q_OP_BYTES: {
+      if (arg < 0 || arg > 4) return VLA_AE_EINVAL;
+      if (arg == 1) {   // attention: prefix K + V of one layer (whole batch)
+        *value = 2LL * d.batch * (long long)std::max(0, H->n_prefix) * d.n_kv_heads * d.head_dim * 2;
+        return VLA_AE_OK;
+      }
+      const OpId id = arg == 0 ? OP_QKV : arg == 2 ? OP_O : arg == 3 ? OP_GU : OP_D;
+      long long b = (long long)H->op[id].O * H->op[id].K * (H->fp8 ? 1 : 2);
+      if (H->fp8) b += 4LL * H->op[id].O;
+      *value = b;
+      return VLA_AE_OK;
+    }
     case VLA_AE_Q_SPLITS:
       *value = H->op[0].S | (H->op[1].S << 8) | (H->op[2].S << 16) | ((long long)H->op[3].S << 24);
       return VLA_AE_OK;
     default:
       return VLA_AE_EINVAL;
   }
+}
+
+int vla_ae_bench_op(vla_ae_t H, int op, int count, int steps, void* stream) {
+  if (!H || op < 0 || op > 4 || count < 1 || steps < 1) return VLA_AE_EINVAL;
+  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+  StepTables* T = nullptr;
+  int rc = get_tables(H, steps, &T);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int parts = ss_parts_of(H, OP_D);
+  for (int i = 0; i < count; ++i) CK(enqueue_op(H, *T, 0, i % H->d.n_layers, op, parts, st));
+  return VLA_AE_OK;
 }
 
 int vla_ae_debug_layer(vla_ae_t H, int layer, int step, int steps, const float* h_in, float* h_out,

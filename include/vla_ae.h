@@ -129,8 +129,19 @@ void vla_ae_destroy(vla_ae_t h);
 #define VLA_AE_Q_KV_BYTES 3           /* bytes of prefix K+V read per step (whole batch) */
 #define VLA_AE_Q_DEVICE_BYTES 4       /* device memory held by the handle */
 #define VLA_AE_Q_SPLITS 5             /* packed split-K of the four GEMMs: qkv | o<<8 | gu<<16 | d<<24 */
+#define VLA_AE_Q_OP_BYTES 6           /* algorithmic bytes one launch of loop kernel `arg` reads from HBM:
+                                         the weight matrix (+ fp8 scales) of op 0 qkv, 2 o, 3 gate/up,
+                                         4 down; the layer's prefix K+V for op 1 (attention) */
 /* Query a property of the handle into *value.  Errors: EINVAL. */
 int vla_ae_query(vla_ae_t h, int what, int arg, long long *value);
+
+/* Benchmark hook: enqueue `count` launches of one kernel of the loop (op: 0 QKV GEMM, 1 attention,
+ * 2 o-projection, 3 gate/up GEMM, 4 down GEMM) for layers 0, 1, 2, ... (cycling), chained by
+ * programmatic dependent launch exactly as inside the loop, with step 0 of the `steps` tables and
+ * the handle's current buffers (the values computed are not meaningful).  Lets a caller time one
+ * kernel with CUDA events on `stream`; weights of successive layers are distinct, so they stream
+ * from HBM.  Asynchronous.  Errors: EINVAL, ENOPREFIX, ECUDA. */
+int vla_ae_bench_op(vla_ae_t h, int op, int count, int steps, void *stream);
 
 /* ------------------------------------------------------------------ test hooks
  * Teacher-forced execution of one DiT layer (per-layer parity): h_in and h_out are device fp32

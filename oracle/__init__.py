@@ -34,7 +34,7 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
 from .model import (  # noqa: F401
     bf16_to_f64, t_schedule, timestep_embedding, silu, rms_norm, modulate, rope_half,
     rope_positions_angles, gqa_attention, linear, swiglu, euler_integrate,
-    adaln_table, dit_layer, velocity, denoise, denoise_batch, OracleWeights,
+    adaln_table, dit_layer, embed_tokens, velocity, denoise, denoise_batch, OracleWeights,
 )
 from .fp8 import (  # noqa: F401
     e4m3_decode, e4m3_encode, quantize_rowwise_e4m3, dequantize_rowwise_e4m3,

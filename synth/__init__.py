@@ -21,8 +21,9 @@ Workload shapes follow the five workloads the action expert is measured on:
 
 Random numbers: numpy's PCG64 bit generator (O'Neill, "PCG: A Family of
 Simple Fast Space-Efficient Statistically Good Algorithms for Random Number
-Generation", 2014) under a ``SeedSequence``.  Weights come from the stream
-``[seed, 0]``; the per-sample inputs of sample ``b`` come from the stream
+Generation", 2014) under a ``SeedSequence``.  Weight matrix number ``i`` in
+canonical order comes from its own stream ``[seed, 0, i]`` (so matrices can be
+drawn in parallel); the per-sample inputs of sample ``b`` come from the stream
 ``[seed, 1, b]``, so a sample's inputs do not depend on the batch it sits in.
 Weights are N(0, 0.02); noise, state and prefix K/V are N(0, 1); all of them
 are drawn in fp32 and rounded to bf16 (round to nearest even), which is how
@@ -150,30 +151,41 @@ def _normal_bf16(rng: np.random.Generator, shape, std: float) -> np.ndarray:
     return out.reshape(shape)
 
 
-def generate_weights(d: Dims, seed: int = 0, std: float = 0.02) -> Dict[str, object]:
-    """All weights as bf16 bit patterns (uint16), drawn in canonical order.
+def _weight_list(d: Dims):
+    """(key, layer or None, shape) in canonical draw order."""
+    sh = weight_shapes(d)
+    items = [("w_in", None), ("b_in", None)]
+    if d.has_state_token:
+        items += [("w_state", None), ("b_state", None)]
+    for l in range(d.n_layers):
+        items += [(name, l) for name in LAYER_WEIGHT_ORDER]
+    items += [(name, None) for name in ("w_fada", "b_fada", "w_out", "b_out")]
+    return [(k, l, sh[k]) for k, l in items]
 
-    Order: in-proj (W, b), state-proj (W, b; only when a state token exists), then per
-    layer adaLN (W, b), q, k, v, o, gate, up, down, then the final adaLN (W, b) and the
+
+def generate_weights(d: Dims, seed: int = 0, std: float = 0.02, threads: int = 8) -> Dict[str, object]:
+    """All weights as bf16 bit patterns (uint16), each matrix from its own seeded stream.
+
+    Canonical order: in-proj (W, b), state-proj (W, b; only when a state token exists), then
+    per layer adaLN (W, b), q, k, v, o, gate, up, down, then the final adaLN (W, b) and the
     out-proj (W, b).  Matrices are ``[out, in]`` row-major.
     """
-    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 0])))
-    sh = weight_shapes(d)
-    w: Dict[str, object] = {}
-    w["w_in"] = _normal_bf16(rng, sh["w_in"], std)
-    w["b_in"] = _normal_bf16(rng, sh["b_in"], std)
-    if d.has_state_token:
-        w["w_state"] = _normal_bf16(rng, sh["w_state"], std)
-        w["b_state"] = _normal_bf16(rng, sh["b_state"], std)
-    layers: List[Dict[str, np.ndarray]] = []
-    for _ in range(d.n_layers):
-        lw = {}
-        for name in LAYER_WEIGHT_ORDER:
-            lw[name] = _normal_bf16(rng, sh[name], std)
-        layers.append(lw)
-    w["layers"] = layers
-    for name in ("w_fada", "b_fada", "w_out", "b_out"):
-        w[name] = _normal_bf16(rng, sh[name], std)
+    from concurrent.futures import ThreadPoolExecutor
+
+    items = _weight_list(d)
+
+    def draw(i):
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 0, i])))
+        return _normal_bf16(rng, items[i][2], std)
+
+    with ThreadPoolExecutor(max_workers=max(1, threads)) as ex:
+        arrays = list(ex.map(draw, range(len(items))))
+    w: Dict[str, object] = {"layers": [dict() for _ in range(d.n_layers)]}
+    for (key, layer, _), a in zip(items, arrays):
+        if layer is None:
+            w[key] = a
+        else:
+            w["layers"][layer][key] = a
     return w
 
 

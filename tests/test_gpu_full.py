@@ -1,0 +1,84 @@
+"""GPU parity at the full workload sizes (StarVLA-shaped, pi0.5-shaped, FP8 pi0.5-shaped), in the
+launch configuration the benchmark times, against the CPU oracle on the same seeded inputs.
+
+The oracle computes every output here (a full loop is a few seconds of BLAS on the host), so
+the comparison covers all actions, plus teacher-forced layers at the first and last Euler step.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import config
+from tests.gpu_util import Case, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device(cuda_device):
+    import __graft_entry__
+    __graft_entry__._build_module().build_library()
+    yield
+
+
+def _teacher_forced(c, step, layers):
+    import torch
+    d = c.d
+    traces = c.oracle_layer_traces(step, d.steps)
+    out = {}
+    for layer in layers:
+        h_in = np.concatenate([traces[b][layer]["h_in"] for b in range(d.batch)])
+        hin = torch.tensor(h_in, dtype=torch.float32, device="cuda")
+        hout = torch.empty_like(hin)
+        c.ae.debug_layer(layer, step, d.steps, hin, hout)
+        torch.cuda.synchronize()
+        ref = np.concatenate([traces[b][layer]["h_out"] for b in range(d.batch)])
+        out[layer] = rel_err(hout.cpu().numpy(), ref)
+    return out
+
+
+@pytest.mark.parametrize("name", ["starvla", "pi05"])
+def test_full_size_bf16(name):
+    c = Case(config(name))
+    try:
+        got = c.denoise()
+        ref = c.oracle_denoise()
+        assert rel_err(got, ref) <= 2e-2
+        L = c.d.n_layers
+        for step in (0, c.d.steps - 1):
+            errs = _teacher_forced(c, step, [0, L // 2, L - 1])
+            assert max(errs.values()) <= 1e-2, (step, errs)
+        # velocity at step 0 (x_0 = noise)
+        import torch
+        x0 = oracle.bf16_to_f64(c.x["noise"])
+        v = torch.empty(x0.shape, dtype=torch.float32, device="cuda")
+        c.ae.debug_velocity(0, c.d.steps, torch.tensor(x0, dtype=torch.float32, device="cuda"), v)
+        noise, st, kp, vp = c.sample_inputs(0)
+        vref = oracle.velocity(noise, 1.0, st, c.W, kp, vp, c.d)
+        assert rel_err(v.cpu().numpy()[0], vref) <= 2e-2
+    finally:
+        c.close()
+
+
+@pytest.mark.parametrize("steps", [1, 10])
+def test_full_size_fp8(steps):
+    c = Case(config("pi05_fp8", steps=steps))
+    try:
+        got = c.denoise()
+        ref_q = c.oracle_denoise()
+        assert rel_err(got, ref_q) <= 2e-2
+        ref_bf16 = c.oracle_denoise(W=oracle.OracleWeights(c.w, c.d, quantized=False))
+        assert rel_err(got, ref_bf16) <= 5e-2
+    finally:
+        c.close()
+
+
+def test_starvla_batch4_sampled():
+    c = Case(config("starvla", batch=4))
+    try:
+        got = c.denoise()
+        ref = c.oracle_denoise(samples=[0, 3])
+        assert rel_err(got[[0, 3]], ref) <= 2e-2
+    finally:
+        c.close()
