@@ -21,10 +21,10 @@ namespace vla {
 constexpr int kAttnThreads = 256;
 
 struct AttnParams {
-  const __nv_bfloat16* q;    // [Ntok][nq][hd]
+  const float* q;            // [Ntok][nq][hd] fp32 (after RoPE)
   const __nv_bfloat16* kc;   // layer K cache [B][nkv][Lpad][hd]
   const __nv_bfloat16* vct;  // layer V^T cache [B][nkv][hd][Lpad]
-  __nv_bfloat16* o_tiles;    // o-proj operand tiles [Nt][KBo][NT][64]
+  __nv_bfloat16* o_tiles;    // o-proj operand tiles [Nt][KBo][2 (hi, lo)][NT][64]
   int nq, nkv, hd, Ts, P, Lpad, Ntok, NT, KBo;
   int S;                     // CTAs per cluster (key chunks), <= 16
   int cs;                    // keys per chunk (multiple of 16)
@@ -51,10 +51,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
   const int g = h / (p.nq / p.nkv);
   const int L = p.P + Ts;
   const int j0 = s * cs, j1 = min(L, j0 + cs), C = max(0, j1 - j0);
-  constexpr int QST = HD + 8, KST = HD + 8;   // padded rows (bf16 elements)
+  constexpr int QST = HD + 4, KST = HD + 8;   // padded rows (q: fp32, K: bf16 elements)
   const int VST = cs + 8;
 
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem);             // [Ts][QST]
+  float* qs = reinterpret_cast<float*>(smem);                              // [Ts][QST]
   __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(smem + p.off_k);   // [cs][KST]
   __nv_bfloat16* vs = reinterpret_cast<__nv_bfloat16*>(smem + p.off_v);   // [HD][VST]
   float* sc = reinterpret_cast<float*>(smem + p.off_s);                    // [Ts][cs]
@@ -81,9 +81,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
   cp_async_commit();
   pdl_wait();
   issue_kv(false);
-  for (int e = tid; e < Ts * (HD / 8); e += kAttnThreads) {
-    const int t = e / (HD / 8), c = e % (HD / 8);
-    cp_async16(qs + t * QST + c * 8, p.q + ((size_t)(b * Ts + t) * p.nq + h) * HD + c * 8);
+  for (int e = tid; e < Ts * (HD / 4); e += kAttnThreads) {
+    const int t = e / (HD / 4), c = e % (HD / 4);
+    cp_async16(qs + t * QST + c * 4, p.q + ((size_t)(b * Ts + t) * p.nq + h) * HD + c * 4);
   }
   cp_async_commit();
   cp_async_wait_all();
@@ -102,8 +102,9 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = min(tg * 4 + i, Ts - 1);
-        float qf[8];
-        bf16x8_to_f32(*reinterpret_cast<const uint4*>(qs + t * QST + c * 8), qf);
+        const float4 q0 = *reinterpret_cast<const float4*>(qs + t * QST + c * 8);
+        const float4 q1 = *reinterpret_cast<const float4*>(qs + t * QST + c * 8 + 4);
+        const float qf[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[i] = fmaf(qf[q], kf[q], acc[i]);
       }
@@ -222,12 +223,24 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
     const int tok = b * Ts + t;
     const int nt = tok / p.NT, row = tok % p.NT;
     const int k = h * HD + d;
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 packed = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-    *reinterpret_cast<uint2*>(p.o_tiles + ((size_t)nt * p.KBo + (k >> 6)) * p.NT * 64 +
-                              sw128_elem_offset(row, k & 63)) = packed;
+    // hi / lo bf16 pair per value, 4 consecutive columns inside one 16-byte chunk
+    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      hi[q] = __float2bfloat16_rn(v[q]);
+      lo[q] = __float2bfloat16_rn(v[q] - __bfloat162float(hi[q]));
+    }
+    __nv_bfloat16* base = p.o_tiles + ((size_t)nt * p.KBo + (k >> 6)) * 2 * p.NT * 64 + sw128_elem_offset(row, k & 63);
+    *reinterpret_cast<uint2*>(base) = *reinterpret_cast<const uint2*>(hi);
+    *reinterpret_cast<uint2*>(base + (size_t)p.NT * 64) = *reinterpret_cast<const uint2*>(lo);
   }
-  if (S > 1) cluster_sync_all(); else __syncthreads();
+  // peers read this CTA's partials: exit only after every CTA has finished reading (the relaxed
+  // arrive does not wait for this CTA's global stores)
+  if (S > 1) {
+    cluster_arrive_relaxed();
+    cluster_wait();
+  }
 }
 
 }  // namespace vla

@@ -1,95 +1,118 @@
 // Skinny weight-streaming GEMM for the action expert's linears, y[t][o] = sum_k W[o][k] x[t][k].
 //
 // Swap-AB: the weight's output rows are the tcgen05 M side (128 rows per tile) and the few
-// tokens (batch x self tokens, padded to a multiple of 16) are the N side, so one M=128 x
+// tokens (batch x self tokens, padded to a multiple of 32) are the N side, so one M=128 x
 // N=NT x K=16 MMA consumes a whole 128-row strip of weights.  At batch 1 the loop is bound by
 // the weight stream from HBM ("跨XPU平台表征视觉-语言-动作模型" section 4.2: the action expert is
 // memory-bound), so the kernel is organised around keeping that stream full:
 //
 //  * weights are pre-packed at create time into 16 KB tiles (128 rows x 64 bf16, or 128 rows x
 //    128 e4m3) already laid out in the 128-byte swizzle the MMA reads, stored [m-tile][k-block]
-//    so every CTA's share is one contiguous range, fetched with 1-D bulk copies (TMA engine);
+//    so every CTA's share is one contiguous range per m-tile, fetched with 1-D bulk copies;
 //  * the producer warp issues those copies before `griddepcontrol.wait`, i.e. while the previous
-//    kernel of the loop is still running (programmatic dependent launch);
+//    kernel of the loop is still running (programmatic dependent launch); 192 threads and
+//    ~110 KB of shared memory let two CTAs share an SM so the overlap really happens;
+//  * the activation operand is a pair of bf16 tiles (hi, lo = x - hi) written by the producing
+//    kernel in the swizzled layout and fetched with one bulk copy; the two tiles are adjacent, so
+//    one MMA with N = 2 NT multiplies both (on B200 an M=128 MMA costs the same ~58 cycles for
+//    any N <= 64) and the epilogue adds the two column halves: the product is fp32-accurate in
+//    the activations while the weights stay exact bf16;
+//  * RMSNorm + adaLN modulate ("AI Infra如何优化VLA" section 算子开发) are applied by linearity:
+//    W (rms(h) (1 + scale) + shift) = rstd * W (h (1 + scale)) + W shift, so producers write
+//    h (1 + scale), this kernel scales by rstd (from partial sums of squares) in the epilogue and
+//    adds the input-independent W shift table;
 //  * split-K across the CTAs of a thread-block cluster, reduced through distributed shared
 //    memory in a fixed order (deterministic, no float atomics);
-//  * fused B-operand prologue (RMSNorm + adaLN modulate of the fp32 residual, "AI Infra如何优化VLA"
-//    section 算子开发) and fused epilogues: RoPE (half-split rotation) writing q and the layer's
-//    K / V^T caches, SwiGLU (section 算子融合) writing the down GEMM's operand, and the gated
-//    residual add writing h plus per-row partial sums of squares for the next RMSNorm.
+//  * fused epilogues: RoPE (half-split rotation) writing q and the layer's K / V^T caches, SwiGLU
+//    (section 算子融合) writing the down GEMM's operand, and the gated residual add writing h,
+//    per-row partial sums of squares and the next GEMM's operand.
 //
-// Warp roles (320 threads): warp 0 = bulk-copy producer, warp 1 = MMA issuer (and TMEM owner),
-// warps 2..9 = math warps (B prologue, fp8 -> bf16 conversion, TMEM read-out, epilogue).
+// Warp roles (192 threads): warp 0 = bulk-copy producer, warp 1 = MMA issuer (and TMEM owner),
+// warps 2..5 = math warps (rstd, fp8 -> bf16 conversion, TMEM read-out, epilogue).
 #pragma once
 #include "ptx.cuh"
 
 namespace vla {
 
 enum EpiKind : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
-enum BMode : int { B_NORM = 0, B_TILES = 1 };
 
-constexpr int kGemmThreads = 320;
-constexpr int kMathThreads = 256;
+constexpr int kGemmThreads = 192;
+constexpr int kMathThreads = 128;
 constexpr int kTileBytes = 16384;      // one packed weight tile
 constexpr int kConvStages = 2;         // fp8 path: converted bf16 A stages (2 x 16 KB each)
+constexpr int kMaxMpc = 4;             // m-tiles per CTA
 
 struct GemmParams {
   // ---- A operand (packed weights)
   const uint8_t* w;        // tiles [Mt][KBt][16 KB]
   const float* wscale;     // fp8: scale per packed row (else nullptr)
   int Mt;                  // 128-row output tiles
+  int mpc;                 // m-tiles per CTA (sharing the activation operand)
   int KBt;                 // weight tiles along K (64 wide for bf16, 128 wide for fp8)
   int K;                   // logical reduction length
   int S;                   // K splits = cluster size along x
   int stages;              // weight-tile ring depth
-  // ---- tokens
+  // ---- tokens / activation operand
   int Ntok;                // valid token rows
-  int NT;                  // token rows per n-tile (multiple of 16, <= 256)
-  int KB;                  // 64-wide k-blocks of the B operand = ceil(K / 64)
-  // ---- B operand
-  const __nv_bfloat16* act;  // B_TILES: [Nt][KB][NT][64] swizzled operand tiles
-  const float* h;            // B_NORM: residual [Ntok][K]
-  const float* ss;           // B_NORM: partial sums of squares [ss_parts][Ntok]
+  int NT;                  // token rows per n-tile (multiple of 32, <= 256)
+  int KB;                  // 64-wide k-blocks of the operand = ceil(K / 64)
+  const __nv_bfloat16* act;  // operand tiles [Nt][KB][2 (hi, lo)][NT][64]
+  // ---- normalised input (QKV, gate/up): y = rstd * acc + cshift
+  const float* ss;           // partial sums of squares of the residual [ss_parts][Ntok]
   int ss_parts;
-  const float* shift;        // B_NORM: [K]
-  const float* scale;        // B_NORM: [K]
-  float eps;
+  const float* cshift;       // [O] = W . shift for this (step, layer)
+  float inv_h, eps;          // 1 / H, RMSNorm epsilon
   // ---- epilogue
   int O;                     // packed output rows
-  float* h_out;              // RESID: residual [Ntok][O] updated in place
+  float* h;                  // RESID: residual [Ntok][O] updated in place
   const float* gate;         // RESID: [O]
-  float* ss_out;             // RESID: [Mt * S][Ntok]
-  __nv_bfloat16* m_out;      // SWIGLU: down-GEMM operand tiles [Nt][KBm][NT][64]
+  float* ss_out;             // RESID: [Mt / mpc * S][Ntok]
+  __nv_bfloat16* b_next;     // RESID: next GEMM's operand tiles [Nt][KBn][2][NT][64] (or nullptr)
+  const float* sc_next;      // RESID: next GEMM's modulation scale [O]
+  int KBn;
+  __nv_bfloat16* m_out;      // SWIGLU: down-GEMM operand tiles [Nt][KBm][2][NT][64]
   int KBm;
-  __nv_bfloat16* q_out;      // QKV: q [Ntok][nq][hd]
+  float* q_out;              // QKV: q [Ntok][nq][hd] fp32
   __nv_bfloat16* kc;         // QKV: layer K cache [B][nkv][Lpad][hd]
   __nv_bfloat16* vct;        // QKV: layer V^T cache [B][nkv][hd][Lpad]
   const float* rope;         // QKV: [Ts][hd/2][2] (cos, sin) for positions P + j
   int nq, nkv, hd, Ts, P, Lpad;
+  const uint8_t* pf_next;     // weights of the next GEMM of the loop: prefetched into L2 (or nullptr)
+  size_t pf_bytes;
   unsigned* status;
   // ---- shared-memory layout (bytes from the 1024-aligned base)
-  int off_b, off_conv, off_bar, off_misc, kmax, smem_bytes;
+  int off_b, off_conv, off_bar, off_misc, off_vec, smem_bytes;
 };
 
-__device__ __forceinline__ void math_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void math_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int EPI, int BMODE, bool FP8>
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __grid_constant__ GemmParams p) {
+// hi/lo bf16 pair of one fp32 value (x = hi + lo to ~2^-16 relative)
+__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+template <int EPI, bool FP8, bool NORM>
+__global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.S;
   const int r = blockIdx.x;          // rank inside the cluster (cluster dims = (S,1,1), grid.x = S)
-  const int mt = blockIdx.y, nt = blockIdx.z;
+  const int mg = blockIdx.y, nt = blockIdx.z;
+  const int mpc = p.mpc;
+  const int mt0 = mg * mpc;
+  const int nmt = min(mpc, p.Mt - mt0);
   const int kt0 = (r * p.KBt) / S, kt1 = ((r + 1) * p.KBt) / S, nkt = kt1 - kt0;
   constexpr int KPT = FP8 ? 2 : 1;   // 64-wide k-blocks per weight tile
   const int kb0 = kt0 * KPT;
   const int kb1 = min(kt1 * KPT, p.KB);
   const int NT = p.NT;
+  const int ntiles = nmt * nkt;      // weight tiles this CTA streams (m-tile major)
 
   uint8_t* sA = smem;                                     // weight ring (and later the reduction buffer)
-  uint8_t* sB = smem + p.off_b;                           // B operand tiles for this CTA's k-range
+  uint8_t* sB = smem + p.off_b;                           // operand tiles (hi, lo) of this CTA's k-range
   uint8_t* sC = smem + p.off_conv;                        // fp8: converted bf16 A stages
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   uint64_t* full = bars;                                  // [stages]
@@ -99,17 +122,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
   uint64_t* cfull = done + 1;                             // [kConvStages]
   uint64_t* cempty = cfull + kConvStages;                 // [kConvStages]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cempty + kConvStages);
-  float* s_shift = reinterpret_cast<float*>(smem + p.off_misc);   // [kmax] modulation slice of this CTA
-  float* s_scale = s_shift + p.kmax;                              // [kmax]
-  float* rpart = s_scale + p.kmax;                                // [256] partial sums of squares
-  float* rstd = rpart + kMathThreads;                             // [NT]
+  float* rpart = reinterpret_cast<float*>(smem + p.off_misc);   // [128] partial sums of squares
+  float* rstd = rpart + kMathThreads;                           // [NT], then [NT][npairs] row sums
+  // per-output-row epilogue vectors of this CTA's rows: W.shift | gate | next scale | fp8 scale
+  float* v_cshift = reinterpret_cast<float*>(smem + p.off_vec);
+  float* v_gate = v_cshift + mpc * 128;
+  float* v_scn = v_gate + mpc * 128;
+  float* v_wsc = v_scn + mpc * 128;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], FP8 ? kMathThreads : 1);
     }
-    mbar_init(bfull, BMODE == B_NORM ? kMathThreads : 1);
+    mbar_init(bfull, 1);
     mbar_init(done, 1);
     for (int i = 0; i < kConvStages; ++i) {
       mbar_init(&cfull[i], kMathThreads);
@@ -117,7 +143,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
     }
     fence_mbar_init();
   }
-  const int tmem_cols = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
+  const bool stacked = 2 * NT <= 256;     // hi and lo rows in one MMA (else two MMAs, N = NT)
+  const int acc_cols = mpc * 2 * NT;      // per m-tile: hi columns [0,NT), lo columns [NT,2NT)
+  const int tmem_cols = acc_cols <= 32 ? 32 : acc_cols <= 64 ? 64 : acc_cols <= 128 ? 128 : acc_cols <= 256 ? 256 : 512;
   if (warp == 1) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
@@ -128,51 +156,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
   const uint32_t tmem_d = *tmem_slot;
   pdl_trigger();
 
+  auto tile_src = [&](int i) {   // i-th weight tile of this CTA: m-tile mt0 + i / nkt, k-tile kt0 + i % nkt
+    return p.w + ((size_t)(mt0 + i / nkt) * p.KBt + kt0 + i % nkt) * kTileBytes;
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer: weight stream
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      const uint8_t* src = p.w + ((size_t)mt * p.KBt + kt0) * kTileBytes;
-      const int prefill = min(nkt, p.stages);
+      const int prefill = min(ntiles, p.stages);
       // the first ring's worth of weights does not depend on the previous kernel
       for (int i = 0; i < prefill; ++i) {
         mbar_arrive_expect_tx(&full[i], kTileBytes);
-        bulk_g2s(sA + (size_t)i * kTileBytes, src + (size_t)i * kTileBytes, kTileBytes, &full[i], pol);
+        bulk_g2s(sA + (size_t)i * kTileBytes, tile_src(i), kTileBytes, &full[i], pol);
       }
-      if (BMODE == B_TILES) {
-        // activation tiles are produced by the previous kernel: only after its completion
-        pdl_wait();
-        const uint32_t bytes = (uint32_t)(kb1 - kb0) * NT * 128u;
-        mbar_arrive_expect_tx(bfull, bytes);
-        bulk_g2s(sB, p.act + ((size_t)nt * p.KB + kb0) * NT * 64, bytes, bfull, policy_evict_last());
+      // the rest of this CTA's weights, then this CTA's slice of the next GEMM's weights, go to
+      // L2 now so HBM keeps streaming while the loop waits on the previous kernel
+      for (int i = prefill; i < ntiles;) {
+        const int j = i / nkt;
+        const int n = min(ntiles, (j + 1) * nkt) - i;   // contiguous run inside one m-tile
+        bulk_prefetch_l2(tile_src(i), (uint32_t)n * kTileBytes);
+        i += n;
       }
-      for (int i = prefill; i < nkt; ++i) {
+      if (p.pf_next) {
+        const size_t nctas = (size_t)gridDim.x * gridDim.y * gridDim.z;
+        const size_t cta = blockIdx.x + (size_t)gridDim.x * (blockIdx.y + (size_t)gridDim.y * blockIdx.z);
+        const size_t chunk = ((p.pf_bytes + nctas - 1) / nctas + 4095) & ~size_t(4095);
+        const size_t b0 = cta * chunk;
+        if (b0 < p.pf_bytes) bulk_prefetch_l2(p.pf_next + b0, (uint32_t)min(chunk, p.pf_bytes - b0));
+      }
+      // activation tiles are produced by the previous kernel: only after its completion
+      pdl_wait();
+      const uint32_t bytes = (uint32_t)(kb1 - kb0) * 2u * NT * 128u;
+      mbar_arrive_expect_tx(bfull, bytes);
+      bulk_g2s(sB, p.act + ((size_t)nt * p.KB + kb0) * 2 * NT * 64, bytes, bfull, policy_evict_last());
+      for (int i = prefill; i < ntiles; ++i) {
         const int s = i % p.stages;
         if (!mbar_wait(&empty[s], ((i / p.stages) - 1) & 1, p.status, DEV_ERR_TIMEOUT_TMA)) break;
         mbar_arrive_expect_tx(&full[s], kTileBytes);
-        bulk_g2s(sA + (size_t)s * kTileBytes, src + (size_t)i * kTileBytes, kTileBytes, &full[s], pol);
+        bulk_g2s(sA + (size_t)s * kTileBytes, tile_src(i), kTileBytes, &full[s], pol);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, NT);
+      const uint32_t idesc = idesc_bf16_f32(128, stacked ? 2 * NT : NT);
       bool ok = mbar_wait(bfull, 0, p.status, DEV_ERR_TIMEOUT_TMA);
       const uint32_t aBase = smem_u32(FP8 ? sC : sA), bBase = smem_u32(sB);
-      uint32_t acc = 0;
-      for (int i = 0; i < nkt && ok; ++i) {
+      const uint32_t bstride = (uint32_t)NT * 128u;   // bytes of one hi or lo tile
+      // one (hi ++ lo) product per K step when stacked, else hi into cols [0,NT), lo into [NT,2NT)
+      auto mma_k = [&](uint32_t d_tmem, uint64_t ad, uint32_t bb, uint32_t acc) {
+        if (stacked) {
+          mma_bf16(d_tmem, ad, sw128_desc(bb), idesc, acc);
+        } else {
+          mma_bf16(d_tmem, ad, sw128_desc(bb), idesc, acc);
+          mma_bf16(d_tmem + (uint32_t)NT, ad, sw128_desc(bb + bstride), idesc, acc);
+        }
+      };
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int j = i / nkt, li = i % nkt;          // accumulator (m-tile), local k-tile
+        const uint32_t d_tmem = tmem_d + (uint32_t)(j * 2 * NT);
         if (!FP8) {
           const int s = i % p.stages;
           ok = mbar_wait(&full[s], (i / p.stages) & 1, p.status, DEV_ERR_TIMEOUT_TMA);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16(tmem_d, sw128_desc(aBase + s * kTileBytes + kk * 32),
-                     sw128_desc(bBase + (uint32_t)i * NT * 128u + kk * 32), idesc, acc);
-            acc = 1;
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_k(d_tmem, sw128_desc(aBase + s * kTileBytes + kk * 32), bBase + (uint32_t)li * 2u * bstride + kk * 32,
+                  (li | kk) != 0);
           mma_commit(&empty[s]);
         } else {
           const int c = i % kConvStages;
@@ -181,14 +234,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
           tc_fence_after();
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            const int lkb = i * 2 + half;                       // local 64-wide k-block
+            const int lkb = li * 2 + half;                      // local 64-wide k-block
             if (kb0 + lkb >= kb1) break;                        // ragged K tail
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_bf16(tmem_d, sw128_desc(aBase + (c * 2 + half) * kTileBytes + kk * 32),
-                       sw128_desc(bBase + (uint32_t)lkb * NT * 128u + kk * 32), idesc, acc);
-              acc = 1;
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_k(d_tmem, sw128_desc(aBase + (c * 2 + half) * kTileBytes + kk * 32),
+                    bBase + (uint32_t)lkb * 2u * bstride + kk * 32, (lkb | kk) != 0);
           }
           mma_commit(&cempty[c]);
         }
@@ -198,7 +249,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
     __syncwarp();
   } else {
     // ------------------------------------------------------------ math warps
-    const int mtid = threadIdx.x - 64;   // 0..255
+    const int mtid = threadIdx.x - 64;   // 0..127
     int conv_done = 0;
     auto convert_one = [&](int i) -> bool {
       // fp8 tile (128 rows x 128 B, swizzled by 16 B chunks) -> two bf16 SW128 tiles
@@ -208,9 +259,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
         return false;
       const uint8_t* src = sA + (size_t)s * kTileBytes;
       uint8_t* dst = sC + (size_t)c * 2 * kTileBytes;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int idx = mtid + j * kMathThreads;   // 0..1023: (row, fp8 chunk)
+#pragma unroll 4
+      for (int jj = 0; jj < 8; ++jj) {
+        const int idx = mtid + jj * kMathThreads;   // 0..1023: (row, fp8 chunk)
         const int row = idx >> 3, ch = idx & 7;
         const uint4 raw = *reinterpret_cast<const uint4*>(src + sw128_chunk_byte(row, ch));
         const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -231,28 +282,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
       mbar_arrive(&empty[s]);
       return true;
     };
+    // the epilogue's per-row vectors are input-independent: stage them before waiting
+    for (int i = mtid; i < nmt * 128; i += kMathThreads) {
+      const int o = mt0 * 128 + i;
+      const bool in = o < p.O;
+      if (NORM) v_cshift[i] = in ? __ldg(p.cshift + o) : 0.f;
+      if (EPI == EPI_RESID) {
+        v_gate[i] = in ? __ldg(p.gate + o) : 0.f;
+        v_scn[i] = (in && p.sc_next) ? __ldg(p.sc_next + o) : 0.f;
+      }
+      if (FP8) v_wsc[i] = in ? __ldg(p.wscale + o) : 0.f;
+    }
     bool ok = true;
     if (FP8) {
       // weights do not depend on the previous kernel: convert the first stages before waiting
-      const int pre = min(nkt, kConvStages);
+      const int pre = min(ntiles, kConvStages);
       for (; conv_done < pre && ok; ++conv_done) ok = convert_one(conv_done);
     }
-    const int nkb = kb1 - kb0;
-    if (BMODE == B_NORM) {
-      // the modulation vectors are input-independent: stage this CTA's slice before waiting
-      for (int i = mtid; i < nkb * 64; i += kMathThreads) {
-        const int k = kb0 * 64 + i;
-        s_shift[i] = k < p.K ? __ldg(p.shift + k) : 0.f;
-        s_scale[i] = k < p.K ? __ldg(p.scale + k) : 0.f;
-      }
-    }
     pdl_wait();
-    if (BMODE == B_NORM) {
+    if (NORM) {
       // rstd per token row from the producers' partial sums of squares: G threads per row each
       // take every G-th part, then the G partials are added in a fixed order (deterministic)
       const int G = NT >= kMathThreads ? 1 : kMathThreads / NT;
-      {
-        const int row = mtid / G, g = mtid % G;
+      for (int base = 0; base < NT; base += kMathThreads / G) {
+        const int row = base + mtid / G, g = mtid % G;
         const int t = nt * NT + row;
         float acc = 0.f;
         if (row < NT && t < p.Ntok) {
@@ -270,174 +323,171 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
           for (; q < p.ss_parts; q += G) acc += __ldcg(p.ss + (size_t)q * p.Ntok + t);
         }
         rpart[mtid] = acc;
-      }
-      math_bar();
-      for (int row = mtid; row < NT; row += kMathThreads) {
-        float acc = 0.f;
-        if (NT >= kMathThreads) {
-          acc = rpart[row];   // G == 1: one thread per row already summed everything
-        } else {
-          for (int g = 0; g < G; ++g) acc += rpart[row * G + g];
+        math_bar();
+        if (mtid < kMathThreads / G) {
+          const int rr = base + mtid;
+          float s2 = 0.f;
+          for (int gg = 0; gg < G; ++gg) s2 += rpart[mtid * G + gg];
+          if (rr < NT) rstd[rr] = rsqrtf(s2 * p.inv_h + p.eps);
         }
-        rstd[row] = rsqrtf(acc / (float)p.K + p.eps);
+        math_bar();
       }
-      math_bar();
-      // u = rms(h) * (1 + scale) + shift -> bf16, written straight into the swizzled B tiles;
-      // loads are issued in batches of 4 chunks so their latencies overlap
-      const int nchunks = NT * nkb * 8;
-      for (int e0 = mtid; e0 < nchunks; e0 += 4 * kMathThreads) {
-        float4 hv[4][2];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = e0 + u * kMathThreads;
-          const int ch = e & 7, rest = e >> 3;
-          const int row = rest % NT, lk = rest / NT;
-          const int t = nt * NT + row;
-          const int k = (kb0 + lk) * 64 + ch * 8;
-          if (e < nchunks && t < p.Ntok && k < p.K) {
-            const float4* hp = reinterpret_cast<const float4*>(p.h + (size_t)t * p.K + k);
-            hv[u][0] = __ldcg(hp);
-            hv[u][1] = __ldcg(hp + 1);
-          } else {
-            hv[u][0] = make_float4(0.f, 0.f, 0.f, 0.f);
-            hv[u][1] = hv[u][0];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int e = e0 + u * kMathThreads;
-          if (e >= nchunks) break;
-          const int ch = e & 7, rest = e >> 3;
-          const int row = rest % NT, lk = rest / NT;
-          const int t = nt * NT + row;
-          const int kl = lk * 64 + ch * 8;
-          const int k = kb0 * 64 + kl;
-          uint4 packed = make_uint4(0, 0, 0, 0);
-          if (t < p.Ntok && k < p.K) {
-            const float rs = rstd[row];
-            const float hvals[8] = {hv[u][0].x, hv[u][0].y, hv[u][0].z, hv[u][0].w,
-                                    hv[u][1].x, hv[u][1].y, hv[u][1].z, hv[u][1].w};
-            uint32_t w4[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float v0 = hvals[2 * q] * rs * (1.f + s_scale[kl + 2 * q]) + s_shift[kl + 2 * q];
-              const float v1 = hvals[2 * q + 1] * rs * (1.f + s_scale[kl + 2 * q + 1]) + s_shift[kl + 2 * q + 1];
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-              w4[q] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-            packed = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-          *reinterpret_cast<uint4*>(sB + (size_t)lk * NT * 128 + sw128_chunk_byte(row, ch)) = packed;
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bfull);
     }
     if (FP8)
-      for (; conv_done < nkt && ok; ++conv_done) ok = convert_one(conv_done);
+      for (; conv_done < ntiles && ok; ++conv_done) ok = convert_one(conv_done);
   }
 
-  // ---------------------------------------------------------------- accumulator -> shared memory
-  float* red = reinterpret_cast<float*>(sA);   // [NT][128] fp32 (weight ring is drained by now)
+  // ---------------------------------------------------------------- accumulators -> shared memory
+  float* red = reinterpret_cast<float*>(sA);   // [mpc][NT][128] fp32 over ring + operand (both consumed)
   if (warp >= 2) {
     const bool ok = mbar_wait(done, 0, p.status, DEV_ERR_TIMEOUT_MMA);
     tc_fence_after();
     const int quarter = warp & 3;            // TMEM lanes this warp may access
-    const int colhalf = (warp - 2) >> 2;     // two warps per lane quarter split the columns
     const int row = quarter * 32 + lane;
-    const int ncol = NT / 2;
-    for (int c0 = colhalf * ncol; c0 < (colhalf + 1) * ncol; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem_d + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0, v);
-      tmem_ld_wait();
+    for (int j = 0; j < nmt; ++j)
+      for (int c0 = 0; c0 < NT; c0 += 16) {
+        float vh[16], vl[16];
+        const uint32_t ta = tmem_d + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(j * 2 * NT + c0);
+        tmem_ld16(ta, vh);
+        tmem_ld16(ta + (uint32_t)NT, vl);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) red[(c0 + j) * 128 + row] = ok ? v[j] : 0.f;
-    }
+        for (int q = 0; q < 16; ++q) red[((size_t)j * NT + c0 + q) * 128 + row] = ok ? vh[q] + vl[q] : 0.f;
+      }
   }
   tc_fence_before();
   if (S > 1) cluster_sync_all(); else __syncthreads();
 
   // ---------------------------------------------------------------- split-K reduction + epilogue
+  // Each math thread owns up to kEpiBatch (pair, column) elements per round; all their remote
+  // partials and global inputs are requested before any is used, so one round costs about one
+  // DSMEM and one L2 latency.
+  constexpr int kEpiBatch = 4;
   if (warp >= 2) {
     const int mtid = threadIdx.x - 64;
-    const int p0 = (r * 64) / S, p1 = ((r + 1) * 64) / S, npairs = p1 - p0;
-    const uint32_t red_local = smem_u32(red);
-    float* sq = reinterpret_cast<float*>(sB);   // [NT][npairs] (B tiles are consumed by now)
-    for (int e = mtid; e < npairs * NT; e += kMathThreads) {
-      const int col = e / npairs, pr = p0 + e % npairs;
-      const int t = nt * NT + col;
-      const int o0 = mt * 128 + 2 * pr;
-      float y0 = 0.f, y1 = 0.f;
-      const uint32_t off = (uint32_t)(col * 128 + 2 * pr) * 4u;
-      if (S > 1) {
-        // all S remote loads in flight first, then the sum in rank order (deterministic)
-        float2 part[16];
+    const int npairs_all = nmt * 64;
+    const int p0 = (r * npairs_all) / S, p1 = ((r + 1) * npairs_all) / S, npairs = p1 - p0;
+    float* sq = rstd + NT;                      // [NT][npairs]
+    const int nel = npairs * NT;
+    for (int e0 = mtid; e0 < nel; e0 += kEpiBatch * kMathThreads) {
+      float2 acc[kEpiBatch];
+      float2 hin[kEpiBatch];
 #pragma unroll
-        for (int s = 0; s < 16; ++s)
-          if (s < S) part[s] = ld_dsmem_f32x2(mapa_shared(red_local + off, (uint32_t)s));
+      for (int u = 0; u < kEpiBatch; ++u) {
+        acc[u] = make_float2(0.f, 0.f);
+        hin[u] = make_float2(0.f, 0.f);
+      }
+      // ---- issue: remote partials (rank order) and the residual rows
 #pragma unroll
-        for (int s = 0; s < 16; ++s)
-          if (s < S) {
-            y0 += part[s].x;
-            y1 += part[s].y;
-          }
-      } else {
-        y0 = red[col * 128 + 2 * pr];
-        y1 = red[col * 128 + 2 * pr + 1];
-      }
-      if (FP8) {
-        if (o0 < p.O) y0 *= p.wscale[o0];
-        if (o0 + 1 < p.O) y1 *= p.wscale[o0 + 1];
-      }
-      const bool valid = (t < p.Ntok) && (o0 < p.O);
-      if (EPI == EPI_RESID) {
-        float hsq = 0.f;
-        if (valid) {
-          float2* hp = reinterpret_cast<float2*>(p.h_out + (size_t)t * p.O + o0);
-          const float2 ho = __ldcg(hp);
-          const float hn0 = ho.x + __ldg(p.gate + o0) * y0;
-          const float hn1 = ho.y + __ldg(p.gate + o0 + 1) * y1;
-          __stcg(hp, make_float2(hn0, hn1));
-          hsq = hn0 * hn0 + hn1 * hn1;
-        }
-        sq[col * npairs + (e % npairs)] = hsq;
-      } else if (EPI == EPI_SWIGLU) {
-        if (valid) {
-          const int j = o0 >> 1;                 // intermediate index: rows (2j, 2j+1) = (gate_j, up_j)
-          const float g = y0;
-          const float m = g / (1.f + __expf(-g)) * y1;
-          const int kb = j >> 6, c = j & 63;
-          p.m_out[((size_t)nt * p.KBm + kb) * NT * 64 + sw128_elem_offset(col, c)] = __float2bfloat16_rn(m);
-        }
-      } else {  // EPI_QKV
-        if (valid) {
-          const int b = t / p.Ts, jt = t % p.Ts;
-          const int qd = p.nq * p.hd, kd = p.nkv * p.hd, half = p.hd >> 1;
-          if (o0 < qd + kd) {
-            const bool isq = o0 < qd;
-            const int local = isq ? o0 : o0 - qd;
-            const int head = local / p.hd, i = (local % p.hd) >> 1;  // pair i rotates (x_i, x_{i+hd/2})
-            const float2 cs = reinterpret_cast<const float2*>(p.rope)[(size_t)jt * half + i];
-            const float r0 = y0 * cs.x - y1 * cs.y;
-            const float r1 = y1 * cs.x + y0 * cs.y;
-            __nv_bfloat16* dst;
-            if (isq) {
-              dst = p.q_out + ((size_t)t * p.nq + head) * p.hd;
-            } else {
-              dst = p.kc + (((size_t)b * p.nkv + head) * p.Lpad + p.P + jt) * p.hd;
+      for (int u = 0; u < kEpiBatch; ++u) {
+        const int e = e0 + u * kMathThreads;
+        if (e >= nel) break;
+        const int col = e / npairs, pr = p0 + e % npairs;
+        const int j = pr >> 6, prj = pr & 63;
+        const size_t roff = ((size_t)j * NT + col) * 128 + 2 * prj;
+        if (S > 1) {
+          const float2* mine = reinterpret_cast<const float2*>(red + roff);
+#pragma unroll
+          for (int s2 = 0; s2 < 16; ++s2)
+            if (s2 < S) {
+              const float2 v = *map_peer(mine, (uint32_t)s2);   // plain loads: batched by the compiler
+              acc[u].x += v.x;
+              acc[u].y += v.y;
             }
-            dst[i] = __float2bfloat16_rn(r0);
-            dst[i + half] = __float2bfloat16_rn(r1);
-          } else {
-            const int local = o0 - qd - kd;
-            const int head = local / p.hd, d = local % p.hd;
-            __nv_bfloat16* dst = p.vct + (((size_t)b * p.nkv + head) * p.hd + d) * p.Lpad + p.P + jt;
-            dst[0] = __float2bfloat16_rn(y0);
-            dst[p.Lpad] = __float2bfloat16_rn(y1);
+        } else {
+          acc[u] = make_float2(red[roff], red[roff + 1]);
+        }
+        if (EPI == EPI_RESID) {
+          const int t = nt * NT + col, o0 = (mt0 + j) * 128 + 2 * prj;
+          if (t < p.Ntok && o0 < p.O) hin[u] = __ldcg(reinterpret_cast<const float2*>(p.h + (size_t)t * p.O + o0));
+        }
+      }
+      // ---- use
+#pragma unroll
+      for (int u = 0; u < kEpiBatch; ++u) {
+        const int e = e0 + u * kMathThreads;
+        if (e >= nel) break;
+        const int col = e / npairs, pl = e % npairs, pr = p0 + pl;
+        const int j = pr >> 6, prj = pr & 63;      // accumulator, pair inside its 128-row tile
+        const int t = nt * NT + col;
+        const int o0 = (mt0 + j) * 128 + 2 * prj;
+        const int lr = o0 - mt0 * 128;            // row inside this CTA's staged vectors
+        float y0 = acc[u].x, y1 = acc[u].y;
+        if (FP8) {
+          y0 *= v_wsc[lr];
+          y1 *= v_wsc[lr + 1];
+        }
+        const bool valid = (t < p.Ntok) && (o0 < p.O);
+        if (NORM && valid) {
+          const float rs = rstd[col];
+          y0 = fmaf(rs, y0, v_cshift[lr]);
+          y1 = fmaf(rs, y1, v_cshift[lr + 1]);
+        }
+        if (EPI == EPI_RESID) {
+          float hsq = 0.f;
+          if (valid) {
+            const float hn0 = fmaf(v_gate[lr], y0, hin[u].x);
+            const float hn1 = fmaf(v_gate[lr + 1], y1, hin[u].y);
+            __stcg(reinterpret_cast<float2*>(p.h + (size_t)t * p.O + o0), make_float2(hn0, hn1));
+            hsq = hn0 * hn0 + hn1 * hn1;
+            if (p.b_next) {
+              __nv_bfloat16 h0, l0, h1, l1;
+              split_bf16(hn0 * (1.f + v_scn[lr]), h0, l0);
+              split_bf16(hn1 * (1.f + v_scn[lr + 1]), h1, l1);
+              const size_t off = operand_offset(t, o0, NT, p.KBn);
+              __nv_bfloat162 hh, ll;
+              hh.x = h0;
+              hh.y = h1;
+              ll.x = l0;
+              ll.y = l1;
+              *reinterpret_cast<__nv_bfloat162*>(p.b_next + off) = hh;
+              *reinterpret_cast<__nv_bfloat162*>(p.b_next + off + (size_t)NT * 64) = ll;
+            }
+          }
+          sq[col * npairs + pl] = hsq;
+        } else if (EPI == EPI_SWIGLU) {
+          if (valid) {
+            const int jj = o0 >> 1;                // intermediate index: rows (2j, 2j+1) = (gate_j, up_j)
+            const float m = y0 / (1.f + __expf(-y0)) * y1;
+            __nv_bfloat16 hi, lo;
+            split_bf16(m, hi, lo);
+            const size_t off = operand_offset(t, jj, NT, p.KBm);
+            p.m_out[off] = hi;
+            p.m_out[off + (size_t)NT * 64] = lo;
+          }
+        } else {  // EPI_QKV
+          if (valid) {
+            const int b = t / p.Ts, jt = t % p.Ts;
+            const int qd = p.nq * p.hd, kd = p.nkv * p.hd, half = p.hd >> 1;
+            if (o0 < qd + kd) {
+              const bool isq = o0 < qd;
+              const int local = isq ? o0 : o0 - qd;
+              const int head = local / p.hd, i = (local % p.hd) >> 1;  // pair i rotates (x_i, x_{i+hd/2})
+              const float2 cs = __ldg(reinterpret_cast<const float2*>(p.rope) + (size_t)jt * half + i);
+              const float r0 = y0 * cs.x - y1 * cs.y;
+              const float r1 = y1 * cs.x + y0 * cs.y;
+              if (isq) {
+                float* dst = p.q_out + ((size_t)t * p.nq + head) * p.hd;
+                dst[i] = r0;
+                dst[i + half] = r1;
+              } else {
+                __nv_bfloat16* dst = p.kc + (((size_t)b * p.nkv + head) * p.Lpad + p.P + jt) * p.hd;
+                dst[i] = __float2bfloat16_rn(r0);
+                dst[i + half] = __float2bfloat16_rn(r1);
+              }
+            } else {
+              const int local = o0 - qd - kd;
+              const int head = local / p.hd, d = local % p.hd;
+              __nv_bfloat16* dst = p.vct + (((size_t)b * p.nkv + head) * p.hd + d) * p.Lpad + p.P + jt;
+              dst[0] = __float2bfloat16_rn(y0);
+              dst[p.Lpad] = __float2bfloat16_rn(y1);
+            }
           }
         }
       }
     }
+    // peers may exit once every CTA has finished reading their partials: arrive now, wait at the end
+    if (S > 1) cluster_arrive_relaxed();
     if (EPI == EPI_RESID) {
       math_bar();
       for (int col = mtid; col < NT; col += kMathThreads) {
@@ -445,12 +495,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_stream_kernel(const __gr
         if (t < p.Ntok) {
           float acc = 0.f;
           for (int q = 0; q < npairs; ++q) acc += sq[col * npairs + q];
-          p.ss_out[(size_t)(mt * S + r) * p.Ntok + t] = acc;
+          p.ss_out[(size_t)(mg * S + r) * p.Ntok + t] = acc;
         }
       }
     }
+  } else if (S > 1) {
+    cluster_arrive_relaxed();
   }
-  if (S > 1) cluster_sync_all(); else __syncthreads();
+  if (S > 1) cluster_wait(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_d, tmem_cols);

@@ -33,10 +33,21 @@ struct TailParams {
   float* x;                 // [B][T][A]
   float* out;               // [B][T][A] copy of x after the update (or nullptr)
   float* v_out;             // [B][T][A] velocity (debug, or nullptr)
+  __nv_bfloat16* b_out_tiles;  // next QKV GEMM's operand tiles [Nt][KBh][2][NT][64]
+  const float* sc_next;     // [H] modulation scale of that GEMM (layer 0 of the next step)
+  int NT, KBh;
   float dt, eps;
   int H, A, T, Ts, has_state, Ntok;
   int do_out, do_in, init_from_noise;
 };
+
+__device__ __forceinline__ void store_operand(__nv_bfloat16* tiles, int t, int k, int NT, int KB, float x) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+  const size_t off = operand_offset(t, k, NT, KB);
+  tiles[off] = hi;
+  tiles[off + (size_t)NT * 64] = lo;
+}
 
 __global__ void __launch_bounds__(kTailThreads) tail_kernel(const __grid_constant__ TailParams p) {
   __shared__ float vsh[kMaxAction];
@@ -100,6 +111,7 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const __grid_constan
     }
     hrow[o] = v;
     sq = fmaf(v, v, sq);
+    store_operand(p.b_out_tiles, t, o, p.NT, p.KBh, v * (1.f + __ldg(p.sc_next + o)));
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
@@ -234,12 +246,18 @@ __global__ void prefix_layout_kernel(const __nv_bfloat16* __restrict__ k, const 
 }
 
 // ---------------------------------------------------------------- debug read-outs
-// ss[t] = sum_k h[t][k]^2 for one row per CTA (fixed-order block reduction)
-__global__ void row_sumsq_kernel(const float* h, float* ss, int H) {
+// ss[t] = sum_k h[t][k]^2 for one row per CTA (fixed-order block reduction), and the row's
+// GEMM operand h (1 + scale) as hi/lo tiles
+__global__ void row_operand_kernel(const float* h, float* ss, __nv_bfloat16* tiles, const float* scale, int H, int NT,
+                                   int KB) {
   __shared__ float red[32];
   const int t = blockIdx.x, tid = threadIdx.x;
   float s = 0.f;
-  for (int k = tid; k < H; k += blockDim.x) s = fmaf(h[(size_t)t * H + k], h[(size_t)t * H + k], s);
+  for (int k = tid; k < H; k += blockDim.x) {
+    const float v = h[(size_t)t * H + k];
+    s = fmaf(v, v, s);
+    store_operand(tiles, t, k, NT, KB, v * (1.f + scale[k]));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if ((tid & 31) == 0) red[tid >> 5] = s;
@@ -250,12 +268,43 @@ __global__ void row_sumsq_kernel(const float* h, float* ss, int H) {
     ss[t] = a;
   }
 }
-// swizzled operand tiles [Nt][KB][NT][64] -> fp32 [Ntok][K]
+// hi/lo operand tiles [Nt][KB][2][NT][64] -> fp32 [Ntok][K] (hi + lo)
 __global__ void untile_kernel(const __nv_bfloat16* tiles, float* out, int Ntok, int K, int NT, int KB) {
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < Ntok * K; e += gridDim.x * blockDim.x) {
     const int t = e / K, k = e % K;
-    const int nt = t / NT, row = t % NT;
-    out[e] = __bfloat162float(tiles[((size_t)nt * KB + (k >> 6)) * NT * 64 + sw128_elem_offset(row, k & 63)]);
+    const size_t off = operand_offset(t, k, NT, KB);
+    out[e] = __bfloat162float(tiles[off]) + __bfloat162float(tiles[off + (size_t)NT * 64]);
+  }
+}
+
+// W . shift for every packed row of one op of one layer and every step:
+// out[k][pr] = sum_c W[pr][c] shift_k[c], with W read back from the packed tiles (fp8: decoded
+// code times the row scale, i.e. exactly the weights the GEMM multiplies).  One warp per row.
+__global__ void cshift_kernel(const uint8_t* __restrict__ wt, const float* __restrict__ wscale, int rows, int KBt,
+                              int K, int fp8, const float* __restrict__ shift, size_t shift_step_stride, int steps,
+                              float* out, size_t out_step_stride) {
+  const int pr = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (pr >= rows) return;
+  const int mt = pr >> 7, r = pr & 127;
+  for (int k = 0; k < steps; ++k) {
+    double acc = 0.0;
+    const float* sh = shift + (size_t)k * shift_step_stride;
+    for (int c = lane; c < K; c += 32) {
+      float w;
+      if (fp8) {
+        const uint8_t* tile = wt + ((size_t)mt * KBt + c / 128) * kTileBytesPack;
+        const uint8_t code = tile[sw128_chunk_byte(r, (c % 128) / 16) + (c % 16)];
+        const uint32_t pair = e4m3x2_to_bf16x2((uint16_t)code);
+        w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&pair)) * wscale[pr];
+      } else {
+        const __nv_bfloat16* tile = reinterpret_cast<const __nv_bfloat16*>(wt + ((size_t)mt * KBt + c / 64) * kTileBytesPack);
+        w = __bfloat162float(tile[sw128_elem_offset(r, c % 64)]);
+      }
+      acc += (double)w * (double)sh[c];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) out[(size_t)k * out_step_stride + pr] = (float)acc;
   }
 }
 __global__ void bf16_to_f32_kernel(const __nv_bfloat16* in, float* out, size_t n) {

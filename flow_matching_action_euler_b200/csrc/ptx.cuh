@@ -107,10 +107,23 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// split cluster barrier: arrive (relaxed: no memory ordering implied) now, wait later
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
   return r;
+}
+// generic pointer to the same shared-memory object in CTA `rank` of the cluster; plain loads
+// through it reach that CTA's shared memory (the compiler may batch them freely)
+template <typename T>
+__device__ __forceinline__ const T* map_peer(const T* p, uint32_t rank) {
+  uint64_t out;
+  asm("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+  return reinterpret_cast<const T*>(out);
 }
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   float v;
@@ -203,6 +216,14 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 // the 16-byte chunk c/8 of row r sits at chunk position (c/8) ^ (r % 8).
 __host__ __device__ __forceinline__ uint32_t sw128_elem_offset(uint32_t r, uint32_t c) {
   return (r >> 3) * 512u + (r & 7u) * 64u + ((((c >> 3) ^ (r & 7u)) & 7u) << 3) + (c & 7u);
+}
+// Element offset of (token t, column k) in activation operand tiles [Nt][KB][2 (hi, lo)][NT][64]:
+// each 64-column block of each n-tile holds a hi tile then a lo tile (NT rows x 128 B each).
+// Add NT * 64 for the lo element.
+__host__ __device__ __forceinline__ size_t operand_offset(int t, int k, int NT, int KB) {
+  const int nt = t / NT, row = t % NT;
+  return ((size_t)nt * KB + (k >> 6)) * 2 * NT * 64 + (row >> 3) * 512u + (row & 7u) * 64u +
+         (((((unsigned)(k & 63) >> 3) ^ (row & 7u)) & 7u) << 3) + (k & 7u);
 }
 // Byte offset of 16-byte chunk `ch` (0..7) of row r.
 __host__ __device__ __forceinline__ uint32_t sw128_chunk_byte(uint32_t r, uint32_t ch) {

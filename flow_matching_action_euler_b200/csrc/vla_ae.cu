@@ -30,7 +30,7 @@ using namespace vla;
 namespace {
 
 constexpr int kMaxDynSmem = 232448;      // 227 KB per CTA on sm_100
-constexpr int kGemmSmemBudget = 116 * 1024;  // leaves room for a second CTA per SM (PDL overlap)
+constexpr int kGemmSmemBudget = 110 * 1024;  // two CTAs (+1 KB reserved each) fit in an SM's 228 KB
 
 #define CK(call)                                                            \
   do {                                                                      \
@@ -48,17 +48,19 @@ size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 enum OpId { OP_QKV = 0, OP_O = 1, OP_GU = 2, OP_D = 3 };
 
 struct OpPlan {
-  int O = 0, K = 0, Mt = 0, KB = 0, KBt = 0, S = 1, stages = 1;
+  int O = 0, K = 0, Mt = 0, KB = 0, KBt = 0, S = 1, stages = 1, mpc = 1;
   size_t wbytes = 0;        // packed tile bytes of one layer
   size_t woff = 0;          // offset inside a layer's packed block
   size_t soff = 0;          // offset of the op's scales inside a layer's scale block (floats)
-  int off_b = 0, off_conv = 0, off_bar = 0, off_misc = 0, kmax = 0, smem = 0;
+  int off_b = 0, off_conv = 0, off_bar = 0, off_misc = 0, off_vec = 0, smem = 0;
 };
 
 struct StepTables {
   int steps = 0;
   float* mod = nullptr;    // [steps][L][6H]
   float* fmod = nullptr;   // [steps][2H]
+  float* cq = nullptr;     // [steps][L][Mt_qkv * 128]: W_qkv . shift_attn
+  float* cg = nullptr;     // [steps][L][Mt_gu * 128]:  W_gu . shift_mlp
   cudaGraphExec_t exec = nullptr;
   int captured_prefix = -1;
 };
@@ -80,9 +82,10 @@ struct vla_ae {
   float* wscale = nullptr;
   __nv_bfloat16 *w_in = nullptr, *b_in = nullptr, *w_st = nullptr, *b_st = nullptr, *w_out = nullptr,
                 *b_out = nullptr, *w_ada = nullptr, *b_ada = nullptr, *w_fada = nullptr, *b_fada = nullptr;
-  __nv_bfloat16 *kc = nullptr, *vct = nullptr, *q = nullptr, *act_o = nullptr, *act_m = nullptr,
+  __nv_bfloat16 *kc = nullptr, *vct = nullptr, *act_x = nullptr, *act_o = nullptr, *act_m = nullptr,
                 *noise_stage = nullptr, *state_stage = nullptr;
-  float *h = nullptr, *ss = nullptr, *x = nullptr, *h_state0 = nullptr, *rope = nullptr, *out_stage = nullptr;
+  float *h = nullptr, *ss = nullptr, *x = nullptr, *h_state0 = nullptr, *rope = nullptr, *out_stage = nullptr,
+        *q = nullptr;
   double* temb = nullptr;
   unsigned* status = nullptr;
   size_t device_bytes = 0;
@@ -143,10 +146,9 @@ using GemmKernel = void (*)(const GemmParams);
 
 GemmKernel gemm_kernel_for(OpId id, bool fp8) {
   switch (id) {
-    case OP_QKV: return fp8 ? gemm_stream_kernel<EPI_QKV, B_NORM, true> : gemm_stream_kernel<EPI_QKV, B_NORM, false>;
-    case OP_O: return fp8 ? gemm_stream_kernel<EPI_RESID, B_TILES, true> : gemm_stream_kernel<EPI_RESID, B_TILES, false>;
-    case OP_GU: return fp8 ? gemm_stream_kernel<EPI_SWIGLU, B_NORM, true> : gemm_stream_kernel<EPI_SWIGLU, B_NORM, false>;
-    default: return fp8 ? gemm_stream_kernel<EPI_RESID, B_TILES, true> : gemm_stream_kernel<EPI_RESID, B_TILES, false>;
+    case OP_QKV: return fp8 ? gemm_stream_kernel<EPI_QKV, true, true> : gemm_stream_kernel<EPI_QKV, false, true>;
+    case OP_GU: return fp8 ? gemm_stream_kernel<EPI_SWIGLU, true, true> : gemm_stream_kernel<EPI_SWIGLU, false, true>;
+    default: return fp8 ? gemm_stream_kernel<EPI_RESID, true, false> : gemm_stream_kernel<EPI_RESID, false, false>;
   }
 }
 
@@ -159,73 +161,107 @@ AttnKernel attn_kernel_for(int hd) {
   }
 }
 
-// shared-memory layout of one GEMM op for a given split / ring depth
+// shared-memory layout of one GEMM op for a given (m-tiles per CTA, split, ring depth)
 void gemm_layout(OpPlan& p, int NT, bool fp8) {
   const int nkt_max = ceil_div(p.KBt, p.S);
   const int nkb_max = std::min(nkt_max * (fp8 ? 2 : 1), p.KB);
-  const size_t a_region = std::max<size_t>((size_t)p.stages * kTileBytes, (size_t)NT * 128 * 4);
-  const size_t b_region = std::max<size_t>((size_t)nkb_max * NT * 128, (size_t)NT * 64 * 4);
+  const size_t b_region = (size_t)2 * nkb_max * NT * 128;
+  const size_t red = (size_t)p.mpc * NT * 128 * 4;        // fp32 accumulators, over ring + operand
+  size_t a_region = (size_t)p.stages * kTileBytes;
+  if (a_region + b_region < red) a_region = red - b_region;
+  a_region = align_up(a_region, 1024);
   const size_t conv = fp8 ? (size_t)kConvStages * 2 * kTileBytes : 0;
   p.off_b = (int)a_region;
-  p.off_conv = (int)(a_region + b_region);
-  p.off_bar = (int)(a_region + b_region + conv);
+  p.off_conv = (int)(a_region + align_up(b_region, 1024));
+  p.off_bar = (int)(p.off_conv + conv);
   const size_t bar_bytes = 8 * (2 * p.stages + 2 + 2 * kConvStages) + 16;
   p.off_misc = (int)(p.off_bar + align_up(bar_bytes, 16));
-  p.kmax = nkb_max * 64;
-  const size_t misc = 4 * (2 * (size_t)p.kmax + kMathThreads + NT);
-  p.smem = (int)(p.off_misc + align_up(misc, 16) + 1024);   // + alignment slack
+  const int npairs_max = ceil_div(p.mpc * 64, p.S);
+  const size_t misc = 4 * ((size_t)kMathThreads + NT + (size_t)NT * npairs_max);
+  p.off_vec = (int)(p.off_misc + align_up(misc, 16));
+  p.smem = (int)(p.off_vec + (size_t)4 * 4 * p.mpc * 128 + 1024);   // + alignment slack
 }
 
-int plan_gemm(vla_ae* H, OpPlan& p, OpId id, int O, int K) {
+bool cluster_fits(GemmKernel kern, const OpPlan& p, int Nt) {
+  if (p.S == 1) return true;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.S, ceil_div(p.Mt, p.mpc), Nt);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = p.smem;
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeClusterDimension;
+  a.val.clusterDim.x = p.S;
+  a.val.clusterDim.y = 1;
+  a.val.clusterDim.z = 1;
+  cfg.attrs = &a;
+  cfg.numAttrs = 1;
+  int nclusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return nclusters >= ceil_div(p.Mt, p.mpc) * Nt;
+}
+
+// Choose m-tiles per CTA and the split so that one wave of CTAs covers the GPU with the
+// fewest weight tiles per CTA, inside the shared-memory budget that keeps two CTAs per SM.
+int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
   const bool fp8 = H->fp8;
-  p.O = O;
-  p.K = K;
-  p.Mt = ceil_div(O, 128);
-  p.KB = ceil_div(K, 64);
-  p.KBt = fp8 ? ceil_div(K, 128) : p.KB;
-  p.wbytes = (size_t)p.Mt * p.KBt * kTileBytes;
-  const int ctas_per_split = p.Mt * H->Nt;
-  int S = std::max(1, std::min({16, p.KBt, H->num_sms / std::max(1, ctas_per_split)}));
+  OpPlan base;
+  base.O = O;
+  base.K = K;
+  base.Mt = ceil_div(O, 128);
+  base.KB = ceil_div(K, 64);
+  base.KBt = fp8 ? ceil_div(K, 128) : base.KB;
+  base.wbytes = (size_t)base.Mt * base.KBt * kTileBytes;
   GemmKernel kern = gemm_kernel_for(id, fp8);
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
-  for (; S >= 1; --S) {
-    p.S = S;
-    // ring depth: as deep as the budget allows (at least 2 when there is more than one tile)
-    const int nkt_max = ceil_div(p.KBt, S);
-    p.stages = 1;
-    gemm_layout(p, H->NT, fp8);
-    const int budget = fp8 ? kMaxDynSmem : kGemmSmemBudget;
-    while (p.stages < std::min(nkt_max, 8)) {
-      OpPlan t = p;
-      t.stages = p.stages + 1;
-      gemm_layout(t, H->NT, fp8);
-      if (t.smem > budget && p.stages >= 2) break;
-      if (t.smem > kMaxDynSmem) break;
-      p = t;
+  // every kernel of the loop asks for the same (maximum) shared-memory carveout, so SMs never
+  // reconfigure between consecutive kernels and a dependent kernel's CTAs can co-reside
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+  const int budget = kGemmSmemBudget;
+  bool found = false;
+  OpPlan best;
+  long best_key = 0;
+  for (int pass = 0; pass < 2 && !found; ++pass) {      // pass 1 allows more than one wave
+    for (int mpc : {1, 2, 4}) {
+      // TMEM: half of it (room for a second CTA per SM), or all of it in the fallback pass
+      if (mpc > base.Mt || mpc * 2 * H->NT > (pass == 0 ? 256 : 512)) continue;
+      const int mg = ceil_div(base.Mt, mpc);
+      for (int S = 1; S <= std::min(16, base.KBt); ++S) {
+        const int ctas = mg * S * H->Nt;
+        if (pass == 0 && ctas > H->num_sms) continue;
+        if (pass == 1 && S > 1 && ctas > H->num_sms) continue;
+        OpPlan p = base;
+        p.mpc = mpc;
+        p.S = S;
+        const int tiles = mpc * ceil_div(base.KBt, S);
+        // deepest ring inside the budget (at least 2 stages when there is more than one tile)
+        p.stages = 1;
+        gemm_layout(p, H->NT, fp8);
+        for (int st = 2; st <= std::min(tiles, 8); ++st) {
+          OpPlan t = p;
+          t.stages = st;
+          gemm_layout(t, H->NT, fp8);
+          if (t.smem > (fp8 ? kMaxDynSmem : budget) && p.stages >= 2) break;
+          if (t.smem > kMaxDynSmem) break;
+          p = t;
+        }
+        if (p.smem > kMaxDynSmem) continue;
+        const int over = p.smem > (fp8 ? kMaxDynSmem : budget) ? 1 : 0;
+        // lexicographic: inside budget, fewest tiles per CTA, smallest split, fewest m-tiles per CTA
+        const long key = (long)over * 1000000 + (long)tiles * 1000 + S * 10 + mpc;
+        if (found && key >= best_key) continue;
+        if (!cluster_fits(kern, p, H->Nt)) continue;
+        best = p;
+        best_key = key;
+        found = true;
+      }
     }
-    if (p.smem > kMaxDynSmem) continue;
-    if (S == 1) break;
-    // the grid must fit in one wave of co-resident clusters
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(S, p.Mt, H->Nt);
-    cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = p.smem;
-    cudaLaunchAttribute a;
-    a.id = cudaLaunchAttributeClusterDimension;
-    a.val.clusterDim.x = S;
-    a.val.clusterDim.y = 1;
-    a.val.clusterDim.z = 1;
-    cfg.attrs = &a;
-    cfg.numAttrs = 1;
-    int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      continue;
-    }
-    if (nclusters >= ctas_per_split) break;
   }
-  if (p.S < 1 || p.smem > kMaxDynSmem) return VLA_AE_EUNSUPPORTED;
+  if (!found) return VLA_AE_EUNSUPPORTED;
+  out = best;
   return VLA_AE_OK;
 }
 
@@ -288,6 +324,7 @@ int plan_attention(vla_ae* H, int P) {
   AttnKernel kern = attn_kernel_for(hd);
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
   // candidate cluster sizes: the preferred one, then smaller, then larger (more, shorter chunks)
   std::vector<int> cands;
   for (int c = S; c >= 1; --c) cands.push_back(c);
@@ -296,7 +333,7 @@ int plan_attention(vla_ae* H, int P) {
     const int cs = (int)align_up((size_t)ceil_div(L, S0), 16);   // keys per chunk, multiple of 16
     const int S = ceil_div(L, cs);
     const int Ts = H->Ts;
-    size_t off = (size_t)Ts * (hd + 8) * 2;
+    size_t off = (size_t)Ts * (hd + 4) * 4;   // q rows, fp32, padded by 16 bytes
     AttnParams a{};
     off = align_up(off, 16);
     a.off_k = (int)off;
@@ -351,12 +388,16 @@ LayerPtrs layer_mod(const vla_ae* H, const StepTables& T, int step, int layer) {
   return {base, base + Hd, base + 2 * Hd, base + 3 * Hd, base + 4 * Hd, base + 5 * Hd};
 }
 
+void set_prefetch(const vla_ae* H, GemmParams& g, OpId id, int layer);
+
 GemmParams gemm_common(const vla_ae* H, OpId id, int layer) {
   const OpPlan& p = H->op[id];
   GemmParams g{};
+  set_prefetch(H, g, id, layer);
   g.w = H->wpack + (size_t)layer * H->layer_wbytes + p.woff;
   g.wscale = H->fp8 ? H->wscale + (size_t)layer * H->layer_scales + p.soff : nullptr;
   g.Mt = p.Mt;
+  g.mpc = p.mpc;
   g.KBt = p.KBt;
   g.K = p.K;
   g.S = p.S;
@@ -365,42 +406,52 @@ GemmParams gemm_common(const vla_ae* H, OpId id, int layer) {
   g.NT = H->NT;
   g.KB = p.KB;
   g.O = p.O;
+  g.inv_h = 1.0f / (float)H->d.hidden;
   g.eps = H->d.rms_eps;
   g.status = H->status;
   g.off_b = p.off_b;
   g.off_conv = p.off_conv;
   g.off_bar = p.off_bar;
   g.off_misc = p.off_misc;
-  g.kmax = p.kmax;
+  g.off_vec = p.off_vec;
   g.smem_bytes = p.smem;
   return g;
 }
 
-cudaError_t launch_gemm(const vla_ae* H, OpId id, const GemmParams& g, cudaStream_t st) {
-  const OpPlan& p = H->op[id];
-  return launch(gemm_kernel_for(id, H->fp8), dim3(p.S, p.Mt, H->Nt), dim3(kGemmThreads), p.smem, st, p.S, true, g);
+// L2 prefetch target of a GEMM: the next GEMM of the loop (QKV -> o -> gate/up -> down -> next QKV)
+void set_prefetch(const vla_ae* H, GemmParams& g, OpId id, int layer) {
+  const OpId next = id == OP_QKV ? OP_O : id == OP_O ? OP_GU : id == OP_GU ? OP_D : OP_QKV;
+  const int nl = id == OP_D ? (layer + 1) % H->d.n_layers : layer;
+  g.pf_next = H->wpack + (size_t)nl * H->layer_wbytes + H->op[next].woff;
+  g.pf_bytes = H->op[next].wbytes;
 }
 
-int ss_parts_of(const vla_ae* H, OpId id) { return H->op[id].Mt * H->op[id].S; }
+cudaError_t launch_gemm(const vla_ae* H, OpId id, const GemmParams& g, cudaStream_t st) {
+  const OpPlan& p = H->op[id];
+  return launch(gemm_kernel_for(id, H->fp8), dim3(p.S, ceil_div(p.Mt, p.mpc), H->Nt), dim3(kGemmThreads), p.smem, st,
+                p.S, true, g);
+}
+
+int ss_parts_of(const vla_ae* H, OpId id) { return ceil_div(H->op[id].Mt, H->op[id].mpc) * H->op[id].S; }
 
 // Kernels of one DiT layer, in loop order.
 enum LayerOp { LOP_QKV = 0, LOP_ATTN = 1, LOP_O = 2, LOP_GU = 3, LOP_D = 4 };
 
 // One kernel of layer `layer` at step `step`.  `ss_in_parts`: partial sums of squares feeding
-// the QKV kernel's RMSNorm (1 after the in-projection, Mt*S of the down GEMM otherwise).
+// the QKV kernel's RMSNorm (1 after the in-projection, those of the down GEMM otherwise).
 cudaError_t enqueue_op(vla_ae* H, const StepTables& T, int step, int layer, int op, int ss_in_parts,
                        cudaStream_t st) {
   const vla_ae_dims& d = H->d;
   const LayerPtrs m = layer_mod(H, T, step, layer);
   const size_t cache = (size_t)layer * d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+  const size_t cl = (size_t)step * d.n_layers + layer;
   switch (op) {
-    case LOP_QKV: {  // RMSNorm + modulate -> QKV -> RoPE -> q, K/V caches
+    case LOP_QKV: {  // (RMSNorm + modulate by linearity) QKV -> RoPE -> q, K/V caches
       GemmParams g = gemm_common(H, OP_QKV, layer);
-      g.h = H->h;
+      g.act = H->act_x;
       g.ss = H->ss;
       g.ss_parts = ss_in_parts;
-      g.shift = m.shift_a;
-      g.scale = m.scale_a;
+      g.cshift = T.cq + cl * H->op[OP_QKV].Mt * 128;
       g.q_out = H->q;
       g.kc = H->kc + cache;
       g.vct = H->vct + cache;
@@ -434,31 +485,38 @@ cudaError_t enqueue_op(vla_ae* H, const StepTables& T, int step, int layer, int 
       return launch(attn_kernel_for(d.head_dim), dim3(H->attn_S, d.n_q_heads, d.batch), dim3(kAttnThreads),
                     H->attn_smem, st, H->attn_S, true, a);
     }
-    case LOP_O: {  // o-projection + gated residual
+    case LOP_O: {  // o-projection + gated residual; writes the gate/up operand h (1 + scale_m)
       GemmParams g = gemm_common(H, OP_O, layer);
       g.act = H->act_o;
-      g.h_out = H->h;
+      g.h = H->h;
       g.gate = m.gate_a;
       g.ss_out = H->ss;
+      g.b_next = H->act_x;
+      g.sc_next = m.scale_m;
+      g.KBn = H->op[OP_GU].KB;
       return launch_gemm(H, OP_O, g, st);
     }
-    case LOP_GU: {  // RMSNorm + modulate -> gate/up -> SwiGLU
+    case LOP_GU: {  // (RMSNorm + modulate by linearity) gate/up -> SwiGLU
       GemmParams g = gemm_common(H, OP_GU, layer);
-      g.h = H->h;
+      g.act = H->act_x;
       g.ss = H->ss;
       g.ss_parts = ss_parts_of(H, OP_O);
-      g.shift = m.shift_m;
-      g.scale = m.scale_m;
+      g.cshift = T.cg + cl * H->op[OP_GU].Mt * 128;
       g.m_out = H->act_m;
       g.KBm = H->op[OP_D].KB;
       return launch_gemm(H, OP_GU, g, st);
     }
-    default: {  // down-projection + gated residual
+    default: {  // down-projection + gated residual; writes the next layer's QKV operand
       GemmParams g = gemm_common(H, OP_D, layer);
       g.act = H->act_m;
-      g.h_out = H->h;
+      g.h = H->h;
       g.gate = m.gate_m;
       g.ss_out = H->ss;
+      if (layer + 1 < d.n_layers) {
+        g.b_next = H->act_x;
+        g.sc_next = layer_mod(H, T, step, layer + 1).scale_a;
+        g.KBn = H->op[OP_QKV].KB;
+      }
       return launch_gemm(H, OP_D, g, st);
     }
   }
@@ -470,7 +528,8 @@ cudaError_t enqueue_layer(vla_ae* H, const StepTables& T, int step, int layer, i
   const size_t cache = (size_t)layer * d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
   cudaError_t e;
   if ((e = enqueue_op(H, T, step, layer, LOP_QKV, ss_in_parts, st)) != cudaSuccess) return e;
-  if (trace && trace->q) bf16_to_f32_kernel<<<64, 256, 0, st>>>(H->q, trace->q, (size_t)H->Ntok * H->qd);
+  if (trace && trace->q)
+    cudaMemcpyAsync(trace->q, H->q, (size_t)H->Ntok * H->qd * 4, cudaMemcpyDeviceToDevice, st);
   if (trace && trace->k && trace->v)
     self_kv_kernel<<<64, 256, 0, st>>>(H->kc + cache, H->vct + cache, trace->k, trace->v, d.batch, H->Ts,
                                        d.n_kv_heads, d.head_dim, H->n_prefix, H->Lpad);
@@ -496,6 +555,9 @@ TailParams tail_common(const vla_ae* H) {
   t.h_state0 = H->h_state0;
   t.noise = H->noise_stage;
   t.x = H->x;
+  t.b_out_tiles = H->act_x;
+  t.NT = H->NT;
+  t.KBh = H->op[OP_QKV].KB;
   t.eps = H->d.rms_eps;
   t.H = H->d.hidden;
   t.A = H->d.action_dim;
@@ -516,6 +578,7 @@ cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
   TailParams t0 = tail_common(H);
   t0.init_from_noise = 1;
   t0.do_in = 1;
+  t0.sc_next = layer_mod(H, T, 0, 0).scale_a;
   cudaError_t e;
   if ((e = launch_tail(H, t0, st)) != cudaSuccess) return e;
   for (int k = 0; k < N; ++k) {
@@ -530,6 +593,7 @@ cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
     t.dt = -1.0f / (float)N;
     t.do_out = 1;
     t.do_in = k + 1 < N;
+    if (t.do_in) t.sc_next = layer_mod(H, T, k + 1, 0).scale_a;
     t.out = k + 1 == N ? H->out_stage : nullptr;
     if ((e = launch_tail(H, t, st)) != cudaSuccess) return e;
   }
@@ -561,6 +625,25 @@ int get_tables(vla_ae* H, int steps, StepTables** out) {
   }
   adaln_table_kernel<<<ceil_div(2 * d.hidden, 8), 256, 0, H->cap>>>(H->w_fada, H->b_fada, c, 2 * d.hidden,
                                                                      d.t_emb_dim, steps, T.fmod, 2 * Hd);
+  CK(cudaGetLastError());
+  // W . shift for the two normalised GEMMs of every (step, layer): RMSNorm's shift by linearity
+  const size_t rq = (size_t)H->op[OP_QKV].Mt * 128, rg = (size_t)H->op[OP_GU].Mt * 128;
+  if ((rc = H->alloc(&T.cq, (size_t)steps * d.n_layers * rq * 4))) return rc;
+  if ((rc = H->alloc(&T.cg, (size_t)steps * d.n_layers * rg * 4))) return rc;
+  for (int l = 0; l < d.n_layers; ++l) {
+    const uint8_t* wl = H->wpack + (size_t)l * H->layer_wbytes;
+    const float* sl = H->fp8 ? H->wscale + (size_t)l * H->layer_scales : nullptr;
+    const float* mod_l = T.mod + (size_t)l * 6 * Hd;
+    const size_t mstep = (size_t)d.n_layers * 6 * Hd;
+    const OpPlan& pq = H->op[OP_QKV];
+    cshift_kernel<<<ceil_div((int)rq, 8), 256, 0, H->cap>>>(wl + pq.woff, sl ? sl + pq.soff : nullptr, (int)rq, pq.KBt,
+                                                           pq.K, H->fp8, mod_l + 0 * Hd, mstep, steps,
+                                                           T.cq + (size_t)l * rq, (size_t)d.n_layers * rq);
+    const OpPlan& pg = H->op[OP_GU];
+    cshift_kernel<<<ceil_div((int)rg, 8), 256, 0, H->cap>>>(wl + pg.woff, sl ? sl + pg.soff : nullptr, (int)rg, pg.KBt,
+                                                           pg.K, H->fp8, mod_l + 3 * Hd, mstep, steps,
+                                                           T.cg + (size_t)l * rg, (size_t)d.n_layers * rg);
+  }
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(H->cap));
   CK(cudaFree(c));
@@ -662,6 +745,7 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   CK(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, H->device));
   if (major != 10) return VLA_AE_EUNSUPPORTED;
   CK(cudaStreamCreateWithFlags(&H->cap, cudaStreamNonBlocking));
+  CK(cudaFuncSetAttribute(tail_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
   H->Ts = d.n_action_tokens + d.has_state_token;
   H->Ntok = d.batch * H->Ts;
   H->Nt = ceil_div(H->Ntok, 256);
@@ -691,9 +775,10 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   const size_t cache = L * B * d.n_kv_heads * (size_t)H->Lpad * d.head_dim;
   if ((rc = H->alloc(&H->kc, cache * 2))) return rc;
   if ((rc = H->alloc(&H->vct, cache * 2))) return rc;
-  if ((rc = H->alloc(&H->q, (size_t)H->Ntok * H->qd * 2))) return rc;
-  if ((rc = H->alloc(&H->act_o, (size_t)H->Nt * H->op[OP_O].KB * H->NT * 64 * 2))) return rc;
-  if ((rc = H->alloc(&H->act_m, (size_t)H->Nt * H->op[OP_D].KB * H->NT * 64 * 2))) return rc;
+  if ((rc = H->alloc(&H->q, (size_t)H->Ntok * H->qd * 4))) return rc;
+  if ((rc = H->alloc(&H->act_x, (size_t)H->Nt * H->op[OP_QKV].KB * 2 * H->NT * 64 * 2))) return rc;
+  if ((rc = H->alloc(&H->act_o, (size_t)H->Nt * H->op[OP_O].KB * 2 * H->NT * 64 * 2))) return rc;
+  if ((rc = H->alloc(&H->act_m, (size_t)H->Nt * H->op[OP_D].KB * 2 * H->NT * 64 * 2))) return rc;
   if ((rc = H->alloc(&H->noise_stage, B * d.n_action_tokens * A * 2))) return rc;
   if ((rc = H->alloc(&H->state_stage, B * A * 2))) return rc;
   if ((rc = H->alloc(&H->h, (size_t)H->Ntok * Hd * 4))) return rc;
@@ -912,8 +997,9 @@ int vla_ae_debug_layer(vla_ae_t H, int layer, int step, int steps, const float* 
   const size_t nh = (size_t)H->Ntok * H->d.hidden;
   cudaStream_t st = H->cap;
   CK(cudaMemcpyAsync(H->h, h_in, nh * 4, cudaMemcpyDeviceToDevice, st));
-  // partial sums of squares of h_in as a single part
-  row_sumsq_kernel<<<H->Ntok, 256, 0, st>>>(H->h, H->ss, H->d.hidden);
+  // sums of squares of h_in (a single part) and the QKV operand h (1 + scale_attn)
+  row_operand_kernel<<<H->Ntok, 256, 0, st>>>(H->h, H->ss, H->act_x, layer_mod(H, *T, step, layer).scale_a,
+                                              H->d.hidden, H->NT, H->op[OP_QKV].KB);
   CK(cudaGetLastError());
   CK(enqueue_layer(H, *T, step, layer, 1, st, trace));
   CK(cudaMemcpyAsync(h_out, H->h, nh * 4, cudaMemcpyDeviceToDevice, st));
@@ -933,6 +1019,7 @@ int vla_ae_debug_velocity(vla_ae_t H, int step, int steps, const float* x, float
   CK(cudaMemcpyAsync(H->x, x, nx * 4, cudaMemcpyDeviceToDevice, st));
   TailParams t0 = tail_common(H);
   t0.do_in = 1;
+  t0.sc_next = layer_mod(H, *T, step, 0).scale_a;
   CK(launch_tail(H, t0, st));
   for (int l = 0; l < d.n_layers; ++l) CK(enqueue_layer(H, *T, step, l, l == 0 ? 1 : ss_parts_of(H, OP_D), st, nullptr));
   TailParams t = tail_common(H);
