@@ -182,7 +182,8 @@ void gemm_layout(OpPlan& p, int NT, bool fp8) {
   p.smem = (int)(p.off_vec + (size_t)4 * 4 * p.mpc * 128 + 1024);   // + alignment slack
 }
 
-bool cluster_fits(GemmKernel kern, const OpPlan& p, int Nt) {
+// one_wave: every cluster of the grid must be co-resident; else at least one cluster must fit
+bool cluster_fits(GemmKernel kern, const OpPlan& p, int Nt, bool one_wave) {
   if (p.S == 1) return true;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.S, ceil_div(p.Mt, p.mpc), Nt);
@@ -200,7 +201,7 @@ bool cluster_fits(GemmKernel kern, const OpPlan& p, int Nt) {
     cudaGetLastError();
     return false;
   }
-  return nclusters >= ceil_div(p.Mt, p.mpc) * Nt;
+  return one_wave ? nclusters >= ceil_div(p.Mt, p.mpc) * Nt : nclusters >= 1;
 }
 
 // Choose m-tiles per CTA and the split so that one wave of CTAs covers the GPU with the
@@ -231,8 +232,7 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
       const int mg = ceil_div(base.Mt, mpc);
       for (int S = 1; S <= std::min(16, base.KBt); ++S) {
         const int ctas = mg * S * H->Nt;
-        if (pass == 0 && ctas > H->num_sms) continue;
-        if (pass == 1 && S > 1 && ctas > H->num_sms) continue;
+        if (pass == 0 && ctas > H->num_sms) continue;   // pass 1: several waves (large batches)
         OpPlan p = base;
         p.mpc = mpc;
         p.S = S;
@@ -253,7 +253,7 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
         // lexicographic: inside budget, fewest tiles per CTA, smallest split, fewest m-tiles per CTA
         const long key = (long)over * 1000000 + (long)tiles * 1000 + S * 10 + mpc;
         if (found && key >= best_key) continue;
-        if (!cluster_fits(kern, p, H->Nt)) continue;
+        if (!cluster_fits(kern, p, H->Nt, pass == 0)) continue;
         best = p;
         best_key = key;
         found = true;
@@ -748,7 +748,9 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   CK(cudaFuncSetAttribute(tail_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
   H->Ts = d.n_action_tokens + d.has_state_token;
   H->Ntok = d.batch * H->Ts;
-  H->Nt = ceil_div(H->Ntok, 256);
+  // token tiles of at most 128 rows: the hi/lo operand pair then fits one MMA (N = 2 NT <= 256)
+  // and a CTA's operand slice stays small enough for shared memory at any K
+  H->Nt = ceil_div(H->Ntok, 128);
   H->NT = (int)align_up(ceil_div(H->Ntok, H->Nt), 32);
   H->qd = d.n_q_heads * d.head_dim;
   H->kd = d.n_kv_heads * d.head_dim;

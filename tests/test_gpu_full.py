@@ -74,11 +74,13 @@ def test_full_size_fp8(steps):
         c.close()
 
 
-def test_starvla_batch4_sampled():
-    c = Case(config("starvla", batch=4))
+@pytest.mark.parametrize("batch", [4, 16, 64])
+def test_starvla_batch_sweep_sampled(batch):
+    c = Case(config("starvla", batch=batch))
     try:
         got = c.denoise()
-        ref = c.oracle_denoise(samples=[0, 3])
-        assert rel_err(got[[0, 3]], ref) <= 2e-2
+        samples = [0, batch - 1]
+        ref = c.oracle_denoise(samples=samples)
+        assert rel_err(got[samples], ref) <= 2e-2
     finally:
         c.close()
