@@ -17,7 +17,7 @@ __all__ = [
     "lib", "VlaAeDims", "VlaAeWeights", "VlaAeTrace", "VlaAeError", "ActionExpert",
     "vla_ae_create", "vla_ae_set_prefix", "vla_ae_denoise", "vla_ae_denoise_host", "vla_ae_status",
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
-    "vla_ae_debug_weight", "vla_ae_bench_op", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
+    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
     "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES",
 ]
 
@@ -77,6 +77,7 @@ vla_ae_debug_layer = _sig("vla_ae_debug_layer", ctypes.c_int, _H, ctypes.c_int, 
 vla_ae_debug_velocity = _sig("vla_ae_debug_velocity", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_debug_weight = _sig("vla_ae_debug_weight", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_bench_op = _sig("vla_ae_bench_op", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P)
+vla_ae_set_prefix_static = _sig("vla_ae_set_prefix_static", ctypes.c_int, _H, _P, _P, ctypes.c_int, _P, _P)
 
 
 class VlaAeError(RuntimeError):
@@ -145,6 +146,11 @@ class ActionExpert:
     def set_prefix(self, k, v, n_prefix: int, state=None, on_device: bool = False, stream=None):
         _check(vla_ae_set_prefix(self.handle, _ptr(k), _ptr(v), int(n_prefix), _ptr(state), int(on_device),
                                  _stream_ptr(stream)), "vla_ae_set_prefix")
+
+    def set_prefix_static(self, k_host, v_host, n_prefix: int, state_host=None, stream=None):
+        """Allocation-free prefix upload from host buffers (see vla_ae_set_prefix_static)."""
+        _check(vla_ae_set_prefix_static(self.handle, _ptr(k_host), _ptr(v_host), int(n_prefix), _ptr(state_host),
+                                        _stream_ptr(stream)), "vla_ae_set_prefix_static")
 
     def denoise(self, noise, steps: int, out, stream=None):
         _check(vla_ae_denoise(self.handle, _ptr(noise), int(steps), _ptr(out), _stream_ptr(stream)),

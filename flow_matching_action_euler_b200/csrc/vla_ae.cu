@@ -17,6 +17,7 @@
 #include <cstring>
 #include <map>
 #include <memory>
+#include <mutex>
 #include <vector>
 
 #include "../../include/vla_ae.h"
@@ -1072,3 +1073,107 @@ int vla_ae_debug_weight(vla_ae_t H, int layer, int which, void* w_host, float* s
 }
 
 }  // extern "C"
+
+// ====================================================================== allocation-free prefix upload
+// Some callers cannot allocate device memory while they run: a robot control loop that must not
+// take the allocator's unbounded latency every cycle, or code that runs while a CUDA graph is
+// being captured on the device (an allocation there is not allowed).  vla_ae_set_prefix with
+// host pointers stages the prefix through cudaMallocAsync'd buffers; vla_ae_set_prefix_static
+// stages it instead, one layer at a time, through this fixed array compiled into the library.
+// Every GPU that loads the library holds the array until the process exits.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // VLA_AE_STATIC_SCRATCH_BYTES
+static __device__ __align__(256) uint8_t g_prefix_scratch[kStaticScratchBytes];
+
+// One layer of the prefix, read from the static staging array: K, V [B][P][nkv][hd] ->
+// the layer's K cache [B][nkv][Lpad][hd] and V^T cache [B][nkv][hd][Lpad].
+__global__ void prefix_layout_static_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                                            __nv_bfloat16* kc, __nv_bfloat16* vct, int B, int P, int nkv, int hd,
+                                            int Lpad) {
+  const size_t total = (size_t)B * P * nkv * hd;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const int d = (int)(e % hd);
+    size_t r = e / hd;
+    const int g = (int)(r % nkv);
+    r /= nkv;
+    const int pp = (int)(r % P);
+    const int b = (int)(r / P);
+    const size_t cache = (size_t)b * nkv + g;
+    kc[(cache * Lpad + pp) * hd + d] = k[e];
+    vct[(cache * hd + d) * Lpad + pp] = v[e];
+  }
+}
+
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[64] = {};   // device address of g_prefix_scratch, per device, set on first use
+
+int static_scratch(int device, uint8_t** out) {
+  if (device < 0 || device >= 64) return VLA_AE_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[device]) {
+    void* p = nullptr;
+    // in host code the array's name only stands for the symbol: ask the runtime for its address
+    cudaError_t e = cudaGetSymbolAddress(&p, g_prefix_scratch);
+    if (e != cudaSuccess || !p) {
+      std::fprintf(stderr, "vla_ae_set_prefix_static: cudaGetSymbolAddress failed: %s\n", cudaGetErrorString(e));
+      return VLA_AE_ECUDA;
+    }
+    g_scratch_ptr[device] = p;
+  }
+  *out = reinterpret_cast<uint8_t*>(g_scratch_ptr[device]);
+  return VLA_AE_OK;
+}
+
+}  // namespace
+
+extern "C" int vla_ae_set_prefix_static(vla_ae_t H, const void* k, const void* v, int n_prefix, const void* state,
+                                        void* stream) {
+  if (!H || n_prefix < 0 || n_prefix > H->d.max_prefix) return VLA_AE_EINVAL;
+  if (n_prefix > 0 && (!k || !v)) return VLA_AE_EINVAL;
+  if (H->d.has_state_token && !state) return VLA_AE_EINVAL;
+  const vla_ae_dims& d = H->d;
+  const size_t per_sample = (size_t)n_prefix * d.n_kv_heads * d.head_dim;   // elements per (sample, layer)
+  const size_t layer_bytes = 2 * (size_t)d.batch * per_sample * 2;         // K and V of one layer, bf16
+  if (layer_bytes > kStaticScratchBytes) {
+    std::fprintf(stderr,
+                 "vla_ae_set_prefix_static: one layer of prefix K+V needs %zu bytes, more than the %zu-byte "
+                 "static staging array (batch * n_prefix * n_kv_heads * head_dim * 4 must be <= %zu)\n",
+                 layer_bytes, kStaticScratchBytes, kStaticScratchBytes);
+    return VLA_AE_EINVAL;
+  }
+  uint8_t* scratch = nullptr;
+  int rc = static_scratch(H->device, &scratch);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (n_prefix != H->n_prefix) {
+    rc = plan_attention(H, n_prefix);
+    if (rc) return rc;
+  }
+  __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(scratch);
+  __nv_bfloat16* vs = ks + (size_t)d.batch * per_sample;
+  const size_t cache_layer = (size_t)d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+  for (int l = 0; l < d.n_layers && per_sample > 0; ++l) {
+    // stream order keeps this layer's copies behind the previous layer's kernel (the array is reused)
+    for (int b = 0; b < d.batch; ++b) {
+      const size_t src = ((size_t)b * d.n_layers + l) * per_sample * 2;   // bytes into [B][L][P][nkv][hd]
+      CK(cudaMemcpyAsync(ks + (size_t)b * per_sample, reinterpret_cast<const uint8_t*>(k) + src, per_sample * 2,
+                         cudaMemcpyHostToDevice, st));
+      CK(cudaMemcpyAsync(vs + (size_t)b * per_sample, reinterpret_cast<const uint8_t*>(v) + src, per_sample * 2,
+                         cudaMemcpyHostToDevice, st));
+    }
+    prefix_layout_static_kernel<<<4 * H->num_sms, 256, 0, st>>>(ks, vs, H->kc + l * cache_layer, H->vct + l * cache_layer,
+                                                                d.batch, n_prefix, d.n_kv_heads, d.head_dim, H->Lpad);
+    CK(cudaGetLastError());
+  }
+  if (d.has_state_token) {
+    CK(cudaMemcpyAsync(H->state_stage, state, (size_t)d.batch * d.action_dim * 2, cudaMemcpyHostToDevice, st));
+    state_proj_kernel<<<dim3(ceil_div(d.hidden, 256), d.batch), 256, 0, st>>>(H->w_st, H->b_st, H->state_stage,
+                                                                               H->h_state0, d.hidden, d.action_dim);
+  }
+  rope_table_kernel<<<ceil_div(H->Ts * d.head_dim / 2, 256), 256, 0, st>>>(reinterpret_cast<float2*>(H->rope), H->Ts,
+                                                                           n_prefix, d.head_dim, (double)d.rope_theta);
+  CK(cudaGetLastError());
+  H->n_prefix = n_prefix;
+  return VLA_AE_OK;
+}

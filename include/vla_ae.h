@@ -99,6 +99,26 @@ int vla_ae_create(const vla_ae_dims *dims, const vla_ae_weights *weights, vla_ae
 int vla_ae_set_prefix(vla_ae_t h, const void *k, const void *v, int n_prefix, const void *state,
                       int on_device, void *stream);
 
+/* Allocation-free variant of vla_ae_set_prefix for host buffers.  The pages have no counterpart:
+ * it exists for callers that cannot allocate device memory while they run, such as a robot control
+ * loop that must not pay the allocator's unbounded latency every cycle, or code running while a
+ * CUDA graph is being captured on the device (an allocation there is not allowed).  Where
+ * vla_ae_set_prefix with host pointers stages the prefix through buffers it allocates, this call
+ * stages it one layer at a time through a fixed device array of VLA_AE_STATIC_SCRATCH_BYTES
+ * (16 MiB) compiled into the library; every GPU that loads the library holds that array until
+ * the process exits.  It allocates nothing and frees nothing.
+ *   k, v   host bf16 [B][L][n_prefix][nkv][hd] (pinned memory gives asynchronous copies);
+ *   state  host bf16 [B][A] (required iff has_state_token).
+ * One layer of K and V for the whole batch, batch * n_prefix * nkv * hd * 4 bytes, must fit in
+ * the array, else VLA_AE_EINVAL (with a message on stderr).  All calls share the one array, which
+ * keeps the last call's contents (nothing in it needs to start at zero): calls that overlap on
+ * the GPU (other streams, other handles on the same device) race on it, so serialise them.  The
+ * first call on a device looks up the array's device address (cudaGetSymbolAddress); make that
+ * first call before any stream capture.  Asynchronous on `stream`.  Errors: EINVAL, ECUDA. */
+#define VLA_AE_STATIC_SCRATCH_BYTES (16u << 20)
+int vla_ae_set_prefix_static(vla_ae_t h, const void *k, const void *v, int n_prefix, const void *state,
+                             void *stream);
+
 /* Run the N-step Euler loop.
  *   noise  device bf16 [B][T][A], the initial x_0;
  *   steps  N >= 1 (t_k = 1 - k/N, dt = -1/N);
