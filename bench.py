@@ -86,6 +86,27 @@ def algorithmic_bytes(d):
     return d.steps * d.n_layers * (wb + d.batch * kv)
 
 
+def replica_seed(rank: int) -> int:
+    """Replicas share the weights and take their own inputs: rank r draws sample inputs with seed r."""
+    return rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's time (the job is done when every replica is done)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput_gbs(bytes_per_loop: int, world: int, ms_per_loop_max: float) -> float:
+    """Whole-job throughput: all replicas' algorithmic bytes over the slowest replica's loop time."""
+    return world * bytes_per_loop / (ms_per_loop_max * 1e-3) / 1e9
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -273,7 +294,7 @@ def run_native(args):
 
     d = workload(args)
     w = generate_weights(d, 0)
-    x = generate_inputs(d, seed=rank)          # each replica its own inputs, same weights
+    x = generate_inputs(d, seed=replica_seed(rank))   # each replica its own inputs, same weights
     ae = fm.ActionExpert(abi_dims(d), w)
     stream = torch.cuda.current_stream()
     kdev = torch.from_numpy(x["k"].view(np.int16)).cuda()
@@ -315,16 +336,12 @@ def run_native(args):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, "cuda")
     if ae.status() != 0:
         raise RuntimeError("device-side timeout during the timed region")
 
     bytes_loop = algorithmic_bytes(d)
-    value = world * bytes_loop / (ms * 1e-3) / 1e9
+    value = job_throughput_gbs(bytes_loop, world, ms)
     kernels_per_loop = ae.query(fm.Q_KERNELS_PER_LOOP, N)
     peak, peak_kind = measured_peak()
     line = {
@@ -387,12 +404,8 @@ def run_native(args):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms_e2e = a.elapsed_time(b) / args.steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        line["e2e"] = {"value": round(world * bytes_loop / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / args.steps, world, "cuda")
+        line["e2e"] = {"value": round(job_throughput_gbs(bytes_loop, world, ms_e2e), 2), "unit": "GB/s",
                        "ms_per_loop": round(ms_e2e, 5),
                        "h2d_bytes_per_step": int(noise_h.numel() * 2),
                        "d2h_bytes_per_step": int(out_h.numel() * 4),

@@ -17,7 +17,7 @@ __all__ = [
     "lib", "VlaAeDims", "VlaAeWeights", "VlaAeTrace", "VlaAeError", "ActionExpert",
     "vla_ae_create", "vla_ae_set_prefix", "vla_ae_denoise", "vla_ae_denoise_host", "vla_ae_status",
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
-    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
+    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
     "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES",
 ]
 
@@ -77,6 +77,7 @@ vla_ae_debug_layer = _sig("vla_ae_debug_layer", ctypes.c_int, _H, ctypes.c_int, 
 vla_ae_debug_velocity = _sig("vla_ae_debug_velocity", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_debug_weight = _sig("vla_ae_debug_weight", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_bench_op = _sig("vla_ae_bench_op", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P)
+vla_ae_debug_wait_probe = _sig("vla_ae_debug_wait_probe", ctypes.c_int, _H, ctypes.c_uint)
 vla_ae_set_prefix_static = _sig("vla_ae_set_prefix_static", ctypes.c_int, _H, _P, _P, ctypes.c_int, _P, _P)
 
 
@@ -180,6 +181,9 @@ class ActionExpert:
 
     def debug_weight(self, layer: int, which: int, w_host, scales_host=None):
         _check(vla_ae_debug_weight(self.handle, layer, which, _ptr(w_host), _ptr(scales_host)), "vla_ae_debug_weight")
+
+    def debug_wait_probe(self, attempts: int):
+        _check(vla_ae_debug_wait_probe(self.handle, int(attempts)), "vla_ae_debug_wait_probe")
 
     def bench_op(self, op: int, count: int, steps: int, stream=None):
         _check(vla_ae_bench_op(self.handle, op, count, steps, _stream_ptr(stream)), "vla_ae_bench_op")

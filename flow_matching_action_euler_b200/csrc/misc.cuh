@@ -245,6 +245,20 @@ __global__ void prefix_layout_kernel(const __nv_bfloat16* __restrict__ k, const 
   }
 }
 
+// ---------------------------------------------------------------- failure-detection probe
+// Waits on an mbarrier that nothing arrives on, with a bounded number of attempts: the wait runs
+// out, the kernel records DEV_ERR_TIMEOUT_MMA in the status word and returns normally.
+__global__ void wait_probe_kernel(unsigned limit, unsigned* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, limit, status, DEV_ERR_TIMEOUT_MMA);
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------- debug read-outs
 // ss[t] = sum_k h[t][k]^2 for one row per CTA (fixed-order block reduction), and the row's
 // GEMM operand h (1 + scale) as hi/lo tiles

@@ -58,6 +58,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   return false;
 }
 
+// Bounded wait with a caller-chosen attempt limit.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, unsigned limit, unsigned* status,
+                                                unsigned err) {
+  for (unsigned i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  if (status) atomicOr(status, err);
+  return false;
+}
+
 // ------------------------------------------------------------------ bulk copies (TMA engine)
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

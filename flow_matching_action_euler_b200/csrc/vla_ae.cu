@@ -989,6 +989,14 @@ int vla_ae_bench_op(vla_ae_t H, int op, int count, int steps, void* stream) {
   return VLA_AE_OK;
 }
 
+int vla_ae_debug_wait_probe(vla_ae_t H, unsigned attempts) {
+  if (!H || attempts == 0 || attempts > (1u << 20)) return VLA_AE_EINVAL;
+  wait_probe_kernel<<<1, 32, 0, H->cap>>>(attempts, H->status);
+  CK(cudaGetLastError());
+  CK(cudaStreamSynchronize(H->cap));
+  return VLA_AE_OK;
+}
+
 int vla_ae_debug_layer(vla_ae_t H, int layer, int step, int steps, const float* h_in, float* h_out,
                        const vla_ae_trace* trace) {
   if (!H || !h_in || !h_out || layer < 0 || layer >= H->d.n_layers || steps < 1 || step < 0 || step >= steps)

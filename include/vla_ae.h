@@ -177,6 +177,12 @@ typedef struct {
 int vla_ae_debug_layer(vla_ae_t h, int layer, int step, int steps, const float *h_in, float *h_out,
                        const vla_ae_trace *trace);
 
+/* Failure-detection probe: run a kernel whose wait on an mbarrier (that nothing arrives on) is
+ * bounded to `attempts` tries (1 .. 2^20).  The wait runs out, the kernel records a timeout in the
+ * handle's device status word and returns; vla_ae_status then reports VLA_AE_ETIMEOUT and the
+ * handle stays usable.  Synchronous.  Errors: EINVAL, ECUDA. */
+int vla_ae_debug_wait_probe(vla_ae_t h, unsigned attempts);
+
 /* v_theta(x, t_step) for device fp32 x [B][T][A] into device fp32 v [B][T][A].  Synchronous. */
 int vla_ae_debug_velocity(vla_ae_t h, int step, int steps, const float *x, float *v);
 

@@ -96,6 +96,8 @@ def test_null_arguments(fm):
     assert fm.vla_ae_debug_layer(None, 0, 0, 1, None, None, None) == fm.EINVAL
     assert fm.vla_ae_debug_velocity(None, 0, 1, None, None) == fm.EINVAL
     assert fm.vla_ae_debug_weight(None, 0, 0, None, None) == fm.EINVAL
+    assert fm.vla_ae_debug_wait_probe(None, 10) == fm.EINVAL
+    assert fm.vla_ae_set_prefix_static(None, None, None, 0, None, None) == fm.EINVAL
     fm.vla_ae_destroy(None)   # no-op
 
 

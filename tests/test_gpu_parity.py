@@ -201,3 +201,15 @@ def test_fp8_tiny():
     ref_bf16 = c.oracle_denoise(W=oracle.OracleWeights(c.w, c.d, quantized=False))
     assert rel_err(got, ref_q) <= 2e-2
     assert rel_err(got, ref_bf16) <= FP8_TOL
+
+
+def test_bounded_wait_reports_timeout_and_handle_stays_usable():
+    """A wait that nothing satisfies runs out, is reported as ETIMEOUT, and nothing hangs."""
+    import flow_matching_action_euler_b200 as fm
+    c = case("tiny")
+    before = c.denoise()
+    c.ae.debug_wait_probe(1000)
+    assert c.ae.status() == fm.ETIMEOUT
+    assert c.ae.status() == fm.OK          # the flag is cleared by reading it
+    after = c.denoise()
+    assert np.array_equal(before, after)
