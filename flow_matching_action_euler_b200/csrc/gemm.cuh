@@ -110,6 +110,14 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
   const int kb1 = min(kt1 * KPT, p.KB);
   const int NT = p.NT;
   const int ntiles = nmt * nkt;      // weight tiles this CTA streams (m-tile major)
+  // split-K epilogue ownership: the nmt * 64 row pairs form octets of 8 pairs; rank q owns octets
+  // [q n8 / S, (q + 1) n8 / S).  An epilogue unit is (token column, owned octet).
+  const int npairs_all = nmt * 64, n8 = npairs_all / 8;
+  const int my_o0 = (r * n8) / S, my_o1 = ((r + 1) * n8) / S;
+  const int my_units = (my_o1 - my_o0) * NT;
+  float4 pre[4];                     // prefetched residual (RESID) or RoPE (QKV) of the first unit
+#pragma unroll
+  for (int q = 0; q < 4; ++q) pre[q] = make_float4(0.f, 0.f, 0.f, 0.f);
 
   uint8_t* sA = smem;                                     // weight ring (and later the reduction buffer)
   uint8_t* sB = smem + p.off_b;                           // operand tiles (hi, lo) of this CTA's k-range
@@ -333,179 +341,259 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
         math_bar();
       }
     }
+    // epilogue inputs that the previous kernel produced (residual rows) or that are static
+    // (RoPE factors): fetch them for this thread's first epilogue unit while the MMAs run
+    if (mtid < my_units) {
+      const int col = mtid % NT, oc = mtid / NT;
+      const int pr0 = (my_o0 + oc) * 8, j = pr0 >> 6;
+      const int t = nt * NT + col;
+      const int o0 = (mt0 + j) * 128 + 2 * (pr0 & 63);
+      if (EPI == EPI_RESID && t < p.Ntok && o0 + 16 <= p.O) {
+        const float4* hp = reinterpret_cast<const float4*>(p.h + (size_t)t * p.O + o0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) pre[q] = __ldcg(hp + q);
+      }
+      if (EPI == EPI_QKV && t < p.Ntok && o0 < p.nq * p.hd + p.nkv * p.hd) {
+        const int local = o0 < p.nq * p.hd ? o0 : o0 - p.nq * p.hd;
+        const int i0 = (local % p.hd) >> 1, half = p.hd >> 1, jt = t % p.Ts;
+        const float4* rp = reinterpret_cast<const float4*>(p.rope + 2 * ((size_t)jt * half + i0));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) pre[q] = __ldg(rp + q);
+      }
+    }
     if (FP8)
       for (; conv_done < ntiles && ok; ++conv_done) ok = convert_one(conv_done);
   }
 
-  // ---------------------------------------------------------------- accumulators -> shared memory
-  float* red = reinterpret_cast<float*>(sA);   // [mpc][NT][128] fp32 over ring + operand (both consumed)
+  // ---------------------------------------------------------------- split-K reduction (push model)
+  // The 64 * nmt row pairs of this CTA's accumulators are partitioned among the S cluster ranks.
+  // Every CTA pushes its partial rows (hi + lo halves already summed) into the owner's receive
+  // buffer with plain stores through distributed shared memory, one cluster barrier makes them
+  // visible, and each owner adds the S partials of its rows from local shared memory in rank
+  // order (deterministic).  No CTA reads another's memory after the barrier, so none waits for
+  // its peers before exiting.  The receive buffer overlays the (drained) weight ring and operand
+  // tiles, so a first barrier makes sure every peer's MMAs are done before anyone writes.
+  const int rmax = 16 * ((n8 + S - 1) / S);            // receive rows per source rank
+  const int RST = NT + 4;                               // padded receive row (floats)
+  float* recv = reinterpret_cast<float*>(sA);           // [S][rmax][RST]
+  float vals[16];
   if (warp >= 2) {
     const bool ok = mbar_wait(done, 0, p.status, DEV_ERR_TIMEOUT_MMA);
     tc_fence_after();
+    (void)ok;
+  }
+  tc_fence_before();
+  if (S > 1) {
+    cluster_arrive_relaxed();   // this CTA's MMAs are complete (or it never had any)
+    cluster_wait();
+  } else {
+    __syncthreads();
+  }
+  if (warp >= 2) {
+    tc_fence_after();
     const int quarter = warp & 3;            // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
-    for (int j = 0; j < nmt; ++j)
+    for (int j = 0; j < nmt; ++j) {
+      const int pr = j * 64 + (row >> 1);
+      const int oct = pr >> 3;
+      const int q = ((oct + 1) * S - 1) / n8;           // owner rank of this row's octet
+      const int q0 = 8 * ((q * n8) / S);                 // first pair owned by q
+      const int lr = 2 * (pr - q0) + (row & 1);
+      float* dst_local = recv + ((size_t)r * rmax + lr) * RST;
+      float* dst = S > 1 ? map_peer_w(dst_local, (uint32_t)q) : dst_local;
       for (int c0 = 0; c0 < NT; c0 += 16) {
-        float vh[16], vl[16];
+        float vl[16];
         const uint32_t ta = tmem_d + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(j * 2 * NT + c0);
-        tmem_ld16(ta, vh);
+        tmem_ld16(ta, vals);
         tmem_ld16(ta + (uint32_t)NT, vl);
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) red[((size_t)j * NT + c0 + q) * 128 + row] = ok ? vh[q] + vl[q] : 0.f;
+        for (int c = 0; c < 16; c += 4)
+          *reinterpret_cast<float4*>(dst + c0 + c) =
+              make_float4(vals[c] + vl[c], vals[c + 1] + vl[c + 1], vals[c + 2] + vl[c + 2], vals[c + 3] + vl[c + 3]);
       }
+    }
   }
   tc_fence_before();
-  if (S > 1) cluster_sync_all(); else __syncthreads();
+  if (S > 1) {
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  } else {
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, tmem_cols);
+  }
 
-  // ---------------------------------------------------------------- split-K reduction + epilogue
-  // Each math thread owns up to kEpiBatch (pair, column) elements per round; all their remote
-  // partials and global inputs are requested before any is used, so one round costs about one
-  // DSMEM and one L2 latency.
-  constexpr int kEpiBatch = 4;
+  // ---------------------------------------------------------------- epilogue on this CTA's rows
   if (warp >= 2) {
     const int mtid = threadIdx.x - 64;
-    const int npairs_all = nmt * 64;
-    const int p0 = (r * npairs_all) / S, p1 = ((r + 1) * npairs_all) / S, npairs = p1 - p0;
-    float* sq = rstd + NT;                      // [NT][npairs]
-    const int nel = npairs * NT;
-    for (int e0 = mtid; e0 < nel; e0 += kEpiBatch * kMathThreads) {
-      float2 acc[kEpiBatch];
-      float2 hin[kEpiBatch];
+    const int noct = my_o1 - my_o0;
+    float* sq = rstd + NT;                      // [NT][noct] partial sums of squares
+    for (int u = mtid; u < my_units; u += kMathThreads) {
+      const int col = u % NT, oc = u / NT;
+      const int pr0 = (my_o0 + oc) * 8;          // first of the unit's 8 row pairs
+      const int j = pr0 >> 6;                    // accumulator (m-tile)
+      const int t = nt * NT + col;
+      const int o0 = (mt0 + j) * 128 + 2 * (pr0 & 63);   // first of 16 output rows
+      const bool valid = (t < p.Ntok) && (o0 < p.O);
+      float y[16];
 #pragma unroll
-      for (int u = 0; u < kEpiBatch; ++u) {
-        acc[u] = make_float2(0.f, 0.f);
-        hin[u] = make_float2(0.f, 0.f);
+      for (int q = 0; q < 16; ++q) y[q] = 0.f;
+      for (int s2 = 0; s2 < S; ++s2) {           // rank order: deterministic
+        const float* rr = recv + ((size_t)s2 * rmax + 16 * oc) * RST + col;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) y[q] += rr[(size_t)q * RST];
       }
-      // ---- issue: remote partials (rank order) and the residual rows
+      const int lr = o0 - mt0 * 128;            // row inside this CTA's staged vectors
+      if (FP8) {
 #pragma unroll
-      for (int u = 0; u < kEpiBatch; ++u) {
-        const int e = e0 + u * kMathThreads;
-        if (e >= nel) break;
-        const int col = e / npairs, pr = p0 + e % npairs;
-        const int j = pr >> 6, prj = pr & 63;
-        const size_t roff = ((size_t)j * NT + col) * 128 + 2 * prj;
-        if (S > 1) {
-          const float2* mine = reinterpret_cast<const float2*>(red + roff);
-#pragma unroll
-          for (int s2 = 0; s2 < 16; ++s2)
-            if (s2 < S) {
-              const float2 v = *map_peer(mine, (uint32_t)s2);   // plain loads: batched by the compiler
-              acc[u].x += v.x;
-              acc[u].y += v.y;
-            }
-        } else {
-          acc[u] = make_float2(red[roff], red[roff + 1]);
-        }
-        if (EPI == EPI_RESID) {
-          const int t = nt * NT + col, o0 = (mt0 + j) * 128 + 2 * prj;
-          if (t < p.Ntok && o0 < p.O) hin[u] = __ldcg(reinterpret_cast<const float2*>(p.h + (size_t)t * p.O + o0));
-        }
+        for (int q = 0; q < 16; ++q) y[q] *= v_wsc[lr + q];
       }
-      // ---- use
+      if (NORM && valid) {
+        const float rs = rstd[col];
 #pragma unroll
-      for (int u = 0; u < kEpiBatch; ++u) {
-        const int e = e0 + u * kMathThreads;
-        if (e >= nel) break;
-        const int col = e / npairs, pl = e % npairs, pr = p0 + pl;
-        const int j = pr >> 6, prj = pr & 63;      // accumulator, pair inside its 128-row tile
-        const int t = nt * NT + col;
-        const int o0 = (mt0 + j) * 128 + 2 * prj;
-        const int lr = o0 - mt0 * 128;            // row inside this CTA's staged vectors
-        float y0 = acc[u].x, y1 = acc[u].y;
-        if (FP8) {
-          y0 *= v_wsc[lr];
-          y1 *= v_wsc[lr + 1];
-        }
-        const bool valid = (t < p.Ntok) && (o0 < p.O);
-        if (NORM && valid) {
-          const float rs = rstd[col];
-          y0 = fmaf(rs, y0, v_cshift[lr]);
-          y1 = fmaf(rs, y1, v_cshift[lr + 1]);
-        }
-        if (EPI == EPI_RESID) {
-          float hsq = 0.f;
-          if (valid) {
-            const float hn0 = fmaf(v_gate[lr], y0, hin[u].x);
-            const float hn1 = fmaf(v_gate[lr + 1], y1, hin[u].y);
-            __stcg(reinterpret_cast<float2*>(p.h + (size_t)t * p.O + o0), make_float2(hn0, hn1));
-            hsq = hn0 * hn0 + hn1 * hn1;
-            if (p.b_next) {
-              __nv_bfloat16 h0, l0, h1, l1;
-              split_bf16(hn0 * (1.f + v_scn[lr]), h0, l0);
-              split_bf16(hn1 * (1.f + v_scn[lr + 1]), h1, l1);
-              const size_t off = operand_offset(t, o0, NT, p.KBn);
-              __nv_bfloat162 hh, ll;
-              hh.x = h0;
-              hh.y = h1;
-              ll.x = l0;
-              ll.y = l1;
-              *reinterpret_cast<__nv_bfloat162*>(p.b_next + off) = hh;
-              *reinterpret_cast<__nv_bfloat162*>(p.b_next + off + (size_t)NT * 64) = ll;
-            }
+        for (int q = 0; q < 16; ++q) y[q] = fmaf(rs, y[q], v_cshift[lr + q]);
+      }
+      const int nv = min(16, p.O - o0);          // valid rows of the unit (RESID rows may end early)
+      float4 in4[4];
+      if (u == mtid && (EPI != EPI_RESID || nv == 16)) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) in4[q] = pre[q];
+      } else if (valid && EPI == EPI_RESID) {
+        float* f = reinterpret_cast<float*>(in4);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) f[q] = q < nv ? __ldcg(p.h + (size_t)t * p.O + o0 + q) : 0.f;
+      } else if (valid && EPI == EPI_QKV && o0 < p.nq * p.hd + p.nkv * p.hd) {
+        const int local = o0 < p.nq * p.hd ? o0 : o0 - p.nq * p.hd;
+        const float4* rp =
+            reinterpret_cast<const float4*>(p.rope + 2 * ((size_t)(t % p.Ts) * (p.hd >> 1) + ((local % p.hd) >> 1)));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) in4[q] = __ldg(rp + q);
+      }
+      const float* in = reinterpret_cast<const float*>(in4);
+      if (EPI == EPI_RESID) {
+        float hsq = 0.f;
+        if (valid) {
+          float hn[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            hn[q] = q < nv ? fmaf(v_gate[lr + q], y[q], in[q]) : 0.f;
+            hsq = fmaf(hn[q], hn[q], hsq);
           }
-          sq[col * npairs + pl] = hsq;
-        } else if (EPI == EPI_SWIGLU) {
-          if (valid) {
-            const int jj = o0 >> 1;                // intermediate index: rows (2j, 2j+1) = (gate_j, up_j)
-            const float m = y0 / (1.f + __expf(-y0)) * y1;
-            __nv_bfloat16 hi, lo;
-            split_bf16(m, hi, lo);
-            const size_t off = operand_offset(t, jj, NT, p.KBm);
-            p.m_out[off] = hi;
-            p.m_out[off + (size_t)NT * 64] = lo;
+          if (nv == 16) {
+            float4* hp = reinterpret_cast<float4*>(p.h + (size_t)t * p.O + o0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              __stcg(hp + q, make_float4(hn[4 * q], hn[4 * q + 1], hn[4 * q + 2], hn[4 * q + 3]));
+          } else {
+            for (int q = 0; q < nv; ++q) __stcg(p.h + (size_t)t * p.O + o0 + q, hn[q]);
           }
-        } else {  // EPI_QKV
-          if (valid) {
-            const int b = t / p.Ts, jt = t % p.Ts;
-            const int qd = p.nq * p.hd, kd = p.nkv * p.hd, half = p.hd >> 1;
-            if (o0 < qd + kd) {
-              const bool isq = o0 < qd;
-              const int local = isq ? o0 : o0 - qd;
-              const int head = local / p.hd, i = (local % p.hd) >> 1;  // pair i rotates (x_i, x_{i+hd/2})
-              const float2 cs = __ldg(reinterpret_cast<const float2*>(p.rope) + (size_t)jt * half + i);
-              const float r0 = y0 * cs.x - y1 * cs.y;
-              const float r1 = y1 * cs.x + y0 * cs.y;
-              if (isq) {
-                float* dst = p.q_out + ((size_t)t * p.nq + head) * p.hd;
-                dst[i] = r0;
-                dst[i + half] = r1;
-              } else {
-                __nv_bfloat16* dst = p.kc + (((size_t)b * p.nkv + head) * p.Lpad + p.P + jt) * p.hd;
-                dst[i] = __float2bfloat16_rn(r0);
-                dst[i + half] = __float2bfloat16_rn(r1);
+          if (p.b_next) {
+            // 16 consecutive columns = two 16-byte chunks of the next operand (hi and lo tiles)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __nv_bfloat16 h0, l0, h1, l1;
+                const int k = 8 * c + 2 * q;
+                split_bf16(hn[k] * (1.f + v_scn[lr + k]), h0, l0);        // zero past the row end
+                split_bf16(hn[k + 1] * (1.f + v_scn[lr + k + 1]), h1, l1);
+                __nv_bfloat162 hh, ll;
+                hh.x = h0;
+                hh.y = h1;
+                ll.x = l0;
+                ll.y = l1;
+                hw[q] = *reinterpret_cast<uint32_t*>(&hh);
+                lw[q] = *reinterpret_cast<uint32_t*>(&ll);
               }
-            } else {
-              const int local = o0 - qd - kd;
-              const int head = local / p.hd, d = local % p.hd;
-              __nv_bfloat16* dst = p.vct + (((size_t)b * p.nkv + head) * p.hd + d) * p.Lpad + p.P + jt;
-              dst[0] = __float2bfloat16_rn(y0);
-              dst[p.Lpad] = __float2bfloat16_rn(y1);
+              const size_t off = operand_offset(t, o0 + 8 * c, NT, p.KBn);
+              *reinterpret_cast<uint4*>(p.b_next + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *reinterpret_cast<uint4*>(p.b_next + off + (size_t)NT * 64) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
+          }
+        }
+        sq[col * noct + oc] = hsq;
+      } else if (EPI == EPI_SWIGLU) {
+        if (valid) {
+          // rows (2j, 2j+1) = (gate_j, up_j): 8 consecutive intermediate indices = one 16-byte chunk
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float g0 = y[4 * q], u0 = y[4 * q + 1], g1 = y[4 * q + 2], u1 = y[4 * q + 3];
+            __nv_bfloat16 h0, l0, h1, l1;
+            split_bf16(g0 / (1.f + __expf(-g0)) * u0, h0, l0);
+            split_bf16(g1 / (1.f + __expf(-g1)) * u1, h1, l1);
+            __nv_bfloat162 hh, ll;
+            hh.x = h0;
+            hh.y = h1;
+            ll.x = l0;
+            ll.y = l1;
+            hw[q] = *reinterpret_cast<uint32_t*>(&hh);
+            lw[q] = *reinterpret_cast<uint32_t*>(&ll);
+          }
+          const size_t off = operand_offset(t, o0 >> 1, NT, p.KBm);
+          *reinterpret_cast<uint4*>(p.m_out + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(p.m_out + off + (size_t)NT * 64) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+      } else {  // EPI_QKV
+        if (valid) {
+          const int b = t / p.Ts, jt = t % p.Ts;
+          const int qd = p.nq * p.hd, kd = p.nkv * p.hd, half = p.hd >> 1;
+          if (o0 < qd + kd) {
+            // 8 rotary pairs (i0 .. i0+7) of one head: x_i in even rows, x_{i+hd/2} in odd rows
+            const bool isq = o0 < qd;
+            const int local = isq ? o0 : o0 - qd;
+            const int head = local / p.hd, i0 = (local % p.hd) >> 1;
+            float r0[8], r1[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float cs = in[2 * q], sn = in[2 * q + 1];
+              r0[q] = y[2 * q] * cs - y[2 * q + 1] * sn;
+              r1[q] = y[2 * q + 1] * cs + y[2 * q] * sn;
+            }
+            if (isq) {
+              float* dst = p.q_out + ((size_t)t * p.nq + head) * p.hd;
+              *reinterpret_cast<float4*>(dst + i0) = make_float4(r0[0], r0[1], r0[2], r0[3]);
+              *reinterpret_cast<float4*>(dst + i0 + 4) = make_float4(r0[4], r0[5], r0[6], r0[7]);
+              *reinterpret_cast<float4*>(dst + i0 + half) = make_float4(r1[0], r1[1], r1[2], r1[3]);
+              *reinterpret_cast<float4*>(dst + i0 + half + 4) = make_float4(r1[4], r1[5], r1[6], r1[7]);
+            } else {
+              __nv_bfloat16* dst = p.kc + (((size_t)b * p.nkv + head) * p.Lpad + p.P + jt) * p.hd;
+              uint32_t a[4], c[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 x0 = __floats2bfloat162_rn(r0[2 * q], r0[2 * q + 1]);
+                __nv_bfloat162 x1 = __floats2bfloat162_rn(r1[2 * q], r1[2 * q + 1]);
+                a[q] = *reinterpret_cast<uint32_t*>(&x0);
+                c[q] = *reinterpret_cast<uint32_t*>(&x1);
+              }
+              *reinterpret_cast<uint4*>(dst + i0) = make_uint4(a[0], a[1], a[2], a[3]);
+              *reinterpret_cast<uint4*>(dst + i0 + half) = make_uint4(c[0], c[1], c[2], c[3]);
+            }
+          } else {
+            const int local = o0 - qd - kd;
+            const int head = local / p.hd, d0 = local % p.hd;
+            __nv_bfloat16* dst = p.vct + (((size_t)b * p.nkv + head) * p.hd + d0) * p.Lpad + p.P + jt;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) dst[(size_t)q * p.Lpad] = __float2bfloat16_rn(y[q]);
           }
         }
       }
     }
-    // peers may exit once every CTA has finished reading their partials: arrive now, wait at the end
-    if (S > 1) cluster_arrive_relaxed();
     if (EPI == EPI_RESID) {
       math_bar();
       for (int col = mtid; col < NT; col += kMathThreads) {
         const int t = nt * NT + col;
         if (t < p.Ntok) {
           float acc = 0.f;
-          for (int q = 0; q < npairs; ++q) acc += sq[col * npairs + q];
+          for (int q = 0; q < noct; ++q) acc += sq[col * noct + q];
           p.ss_out[(size_t)(mg * S + r) * p.Ntok + t] = acc;
         }
       }
     }
-  } else if (S > 1) {
-    cluster_arrive_relaxed();
-  }
-  if (S > 1) cluster_wait(); else __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_d, tmem_cols);
   }
 }
 

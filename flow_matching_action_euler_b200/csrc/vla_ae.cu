@@ -167,7 +167,8 @@ void gemm_layout(OpPlan& p, int NT, bool fp8) {
   const int nkt_max = ceil_div(p.KBt, p.S);
   const int nkb_max = std::min(nkt_max * (fp8 ? 2 : 1), p.KB);
   const size_t b_region = (size_t)2 * nkb_max * NT * 128;
-  const size_t red = (size_t)p.mpc * NT * 128 * 4;        // fp32 accumulators, over ring + operand
+  // split-K receive buffer [S][16 ceil(8 mpc / S)][NT + 4] fp32, over ring + operand
+  const size_t red = (size_t)p.S * 16 * ceil_div(8 * p.mpc, p.S) * (NT + 4) * 4;
   size_t a_region = (size_t)p.stages * kTileBytes;
   if (a_region + b_region < red) a_region = red - b_region;
   a_region = align_up(a_region, 1024);
@@ -177,8 +178,8 @@ void gemm_layout(OpPlan& p, int NT, bool fp8) {
   p.off_bar = (int)(p.off_conv + conv);
   const size_t bar_bytes = 8 * (2 * p.stages + 2 + 2 * kConvStages) + 16;
   p.off_misc = (int)(p.off_bar + align_up(bar_bytes, 16));
-  const int npairs_max = ceil_div(p.mpc * 64, p.S);
-  const size_t misc = 4 * ((size_t)kMathThreads + NT + (size_t)NT * npairs_max);
+  const int noct_max = ceil_div(p.mpc * 8, p.S);        // octets of 8 row pairs per rank
+  const size_t misc = 4 * ((size_t)kMathThreads + NT + (size_t)NT * noct_max);
   p.off_vec = (int)(p.off_misc + align_up(misc, 16));
   p.smem = (int)(p.off_vec + (size_t)4 * 4 * p.mpc * 128 + 1024);   // + alignment slack
 }
