@@ -1,245 +1,269 @@
-// GQA attention of the action tokens over the cached VLM prefix plus themselves (no mask).
+// GQA attention of the action tokens over the cached VLM prefix plus themselves (no mask), on
+// the tensor cores.
 //
-// One cluster per (sample b, q head h); its CTAs split the keys (prefix followed by the self
-// tokens) into chunks of `cs` keys (a multiple of 16).  Each CTA stages its K rows, V^T columns
-// and q with 16-byte cp.async copies, computes scores, a warp-shuffle softmax with its local
-// max / sum, and a partial P.V; the CTAs then merge their partials through distributed shared
-// memory in a fixed order (max-rescaled sums, as in split-K "flash decoding").  The prefix part
-// of K / V^T does not depend on the previous kernel and is copied before `griddepcontrol.wait`;
-// the self part (written by the QKV epilogue) and q after it.  The merged output is written as
-// bf16 straight into the o-projection's operand tiles.
+// The rep = nq / nkv query heads that share kv head g are stacked into one row set of
+// R = rep * Ts rows (row = head_in_group * Ts + token), cut into blocks of 64 rows.  One
+// cluster per (sample, kv head, row block); its CTAs split the keys (prefix then self tokens)
+// into spans; a CTA walks its span in sub-chunks of CS keys.  Each CTA: 4 warps x 16 rows,
+// S = Q K^T with mma.sync m16n8k16 (bf16 in, fp32 accumulate), online exp2 softmax over the
+// sub-chunks (row max and sum via quad shuffles, running rescale of the accumulators),
+// O += P V with P re-packed from the score registers, then every CTA pushes
+// (row max, row sum, partial O) of each row into the shared memory of the row's owner CTA;
+// after one cluster barrier owners merge the chunks in rank order (max-rescaled sums, as in
+// split-KV "flash decoding") and write the o-projection's hi/lo operand tiles.
+// K and V^T of the prefix are static during the loop and are copied before
+// `griddepcontrol.wait`; the self rows (written by the QKV epilogue) and q after it.
 //
-// Kept on CUDA cores: at batch 1 the whole attention is ~1-3% of the loop's bytes
-// ("AI Infra如何优化VLA" section 算子开发 keeps SDPA on a library kernel for the same reason).
-// Row strides are padded by 16 bytes so that 16-byte shared loads of consecutive rows hit
-// distinct banks.
+// The pages keep SDPA on a library kernel ("AI Infra如何优化VLA" section 算子开发); here it is a
+// hand-written kernel.  At batch 1 attention reads 1-3 % of the loop's bytes but sits on the
+// critical path once per layer, so the kernel is built for latency: few, short CTAs.
 #pragma once
 #include "ptx.cuh"
 
 namespace vla {
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 128;
+constexpr int kAttnRows = 64;   // query rows per CTA (4 warps x 16)
 
 struct AttnParams {
-  const float* q;            // [Ntok][nq][hd] fp32 (after RoPE)
+  const __nv_bfloat16* q;    // [B][nkv][Rpad][hd] bf16, row = head_in_group * Ts + token (after RoPE)
   const __nv_bfloat16* kc;   // layer K cache [B][nkv][Lpad][hd]
   const __nv_bfloat16* vct;  // layer V^T cache [B][nkv][hd][Lpad]
   __nv_bfloat16* o_tiles;    // o-proj operand tiles [Nt][KBo][2 (hi, lo)][NT][64]
   int nq, nkv, hd, Ts, P, Lpad, Ntok, NT, KBo;
   int S;                     // CTAs per cluster (key chunks), <= 16
-  int cs;                    // keys per chunk (multiple of 16)
+  int span;                  // keys per CTA (multiple of 16); CTA c takes [c span, min(L, (c+1) span))
+  int nrb;                   // 64-row blocks per kv head
+  int Rpad;                  // nrb * 64
+  int rpo;                   // rows owned per CTA in the merge = ceil(64 / S)
   float scale;               // 1 / sqrt(hd)
-  int off_k, off_v, off_s, off_o, off_ml, smem_bytes;
+  int off_k, off_v, off_recv, smem_bytes;
 };
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
+__device__ __forceinline__ void ldsm_x4(const void* smem_row_addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(smem_u32(smem_row_addr)));
+}
+__device__ __forceinline__ void mma_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int HD>
+template <int HD, int CS>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int QST = HD + 8, KST = HD + 8, VST = CS + 8;   // padded rows (bf16): conflict-free ldmatrix
+  constexpr int RST = HD + 4;                                 // receive row: O[HD], max, sum
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int S = p.S, cs = p.cs, Ts = p.Ts;
-  const int g = h / (p.nq / p.nkv);
+  const int g4 = lane >> 2, t4 = lane & 3;
+  const int c = blockIdx.x, rb = blockIdx.y % p.nrb, kvh = blockIdx.y / p.nrb, b = blockIdx.z;
+  const int S = p.S, Ts = p.Ts;
   const int L = p.P + Ts;
-  const int j0 = s * cs, j1 = min(L, j0 + cs), C = max(0, j1 - j0);
-  constexpr int QST = HD + 4, KST = HD + 8;   // padded rows (q: fp32, K: bf16 elements)
-  const int VST = cs + 8;
+  const int kbeg = c * p.span, kend = min(L, kbeg + p.span);   // this CTA's keys (>= 1 of them)
+  const int nch = (kend - kbeg + CS - 1) / CS;
+  const int rep = p.nq / p.nkv, R = rep * Ts;
 
-  float* qs = reinterpret_cast<float*>(smem);                              // [Ts][QST]
-  __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(smem + p.off_k);   // [cs][KST]
-  __nv_bfloat16* vs = reinterpret_cast<__nv_bfloat16*>(smem + p.off_v);   // [HD][VST]
-  float* sc = reinterpret_cast<float*>(smem + p.off_s);                    // [Ts][cs]
-  float* po = reinterpret_cast<float*>(smem + p.off_o);                    // [Ts][HD] partial O
-  float* ml = reinterpret_cast<float*>(smem + p.off_ml);                   // m[Ts], l[Ts], weights[16][Ts]
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem);              // [64][QST]
+  __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(smem + p.off_k);    // [CS][KST]
+  __nv_bfloat16* vs = reinterpret_cast<__nv_bfloat16*>(smem + p.off_v);    // [HD][VST]
+  float* recv = reinterpret_cast<float*>(smem + p.off_recv);               // [S][rpo][RST]
 
   pdl_trigger();
-  const __nv_bfloat16* kbase = p.kc + ((size_t)b * p.nkv + g) * p.Lpad * HD;
-  const __nv_bfloat16* vbase = p.vct + ((size_t)b * p.nkv + g) * (size_t)HD * p.Lpad;
-  const int nvc = (C + 7) >> 3;   // 16-byte chunks per V^T row
-  auto issue_kv = [&](bool prefix_part) {
-    for (int e = tid; e < C * (HD / 8); e += kAttnThreads) {
-      const int jj = j0 + e / (HD / 8), c = e % (HD / 8);
-      if ((jj < p.P) == prefix_part) cp_async16(ks + (jj - j0) * KST + c * 8, kbase + (size_t)jj * HD + c * 8);
+  const __nv_bfloat16* kbase = p.kc + ((size_t)b * p.nkv + kvh) * p.Lpad * HD;
+  const __nv_bfloat16* vbase = p.vct + ((size_t)b * p.nkv + kvh) * (size_t)HD * p.Lpad;
+  // K rows and V^T columns of sub-chunk j0 (part = 0: prefix only, 1: self only, 2: all).  The
+  // spans are multiples of 16 keys, so an 8-column V^T copy never crosses into the next CTA's
+  // keys; copies past L stay inside the Lpad-long cache rows and meet P = 0.
+  auto issue_kv = [&](int j0, int part) {
+    for (int e = tid; e < CS * (HD / 8); e += kAttnThreads) {
+      const int jj = j0 + e / (HD / 8), cc = e % (HD / 8);
+      if (jj < kend && (part == 2 || (jj < p.P) == (part == 0)))
+        cp_async16(ks + (jj - j0) * KST + cc * 8, kbase + (size_t)jj * HD + cc * 8);
     }
-    for (int e = tid; e < HD * nvc; e += kAttnThreads) {
-      const int d = e / nvc, c = e % nvc;
-      const int key0 = j0 + c * 8;
-      if ((key0 + 8 <= p.P) == prefix_part) cp_async16(vs + d * VST + c * 8, vbase + (size_t)d * p.Lpad + key0);
+    for (int e = tid; e < HD * (CS / 8); e += kAttnThreads) {
+      const int d = e / (CS / 8), cc = e % (CS / 8);
+      const int key0 = j0 + cc * 8;
+      if (key0 < kend) {
+        if (part == 2 || (key0 + 8 <= p.P) == (part == 0))
+          cp_async16(vs + d * VST + cc * 8, vbase + (size_t)d * p.Lpad + key0);
+      } else if (part != 1) {   // zero columns past the CTA's keys: P is 0 there, V must be finite
+        *reinterpret_cast<uint4*>(vs + d * VST + cc * 8) = make_uint4(0, 0, 0, 0);
+      }
     }
   };
-  // prefix keys are static during the loop: fetch them before waiting on the QKV kernel
-  issue_kv(true);
+  issue_kv(kbeg, 0);
   cp_async_commit();
   pdl_wait();
-  issue_kv(false);
-  for (int e = tid; e < Ts * (HD / 4); e += kAttnThreads) {
-    const int t = e / (HD / 4), c = e % (HD / 4);
-    cp_async16(qs + t * QST + c * 4, p.q + ((size_t)(b * Ts + t) * p.nq + h) * HD + c * 4);
+  issue_kv(kbeg, 1);
+  const __nv_bfloat16* qbase = p.q + (((size_t)b * p.nkv + kvh) * p.Rpad + (size_t)rb * kAttnRows) * HD;
+  for (int e = tid; e < kAttnRows * (HD / 8); e += kAttnThreads) {
+    const int r = e / (HD / 8), cc = e % (HD / 8);
+    cp_async16(qs + r * QST + cc * 8, qbase + (size_t)r * HD + cc * 8);
   }
   cp_async_commit();
-  cp_async_wait_all();
-  __syncthreads();
 
-  // scores: item = (key, group of 4 tokens); 8 dims per 16-byte load
-  const int ntg = (Ts + 3) >> 2;
-  for (int it = tid; it < ntg * C; it += kAttnThreads) {
-    const int jj = it % C, tg = it / C;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint4* kr = reinterpret_cast<const uint4*>(ks + jj * KST);
-#pragma unroll 2
-    for (int c = 0; c < HD / 8; ++c) {
-      float kf[8];
-      bf16x8_to_f32(kr[c], kf);
+  const float sl2 = p.scale * 1.4426950408889634f;   // 1/sqrt(hd) * log2(e)
+  const int arow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows g4 and g4 + 8 of the warp
+  float oacc[HD / 8][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = min(tg * 4 + i, Ts - 1);
-        const float4 q0 = *reinterpret_cast<const float4*>(qs + t * QST + c * 8);
-        const float4 q1 = *reinterpret_cast<const float4*>(qs + t * QST + c * 8 + 4);
-        const float qf[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+  for (int n = 0; n < HD / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+
+  for (int ch = 0; ch < nch; ++ch) {
+    const int j0 = kbeg + ch * CS, C = min(CS, kend - j0);
+    if (ch > 0) {
+      __syncthreads();   // every warp is done with the previous sub-chunk
+      issue_kv(j0, 2);
+      cp_async_commit();
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    // S = Q K^T for the warp's 16 rows
+    float sacc[CS / 8][4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[i] = fmaf(qf[q], kf[q], acc[i]);
+    for (int j = 0; j < CS / 8; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.f;
+#pragma unroll 4
+    for (int kst = 0; kst < HD / 16; ++kst) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(qs + arow * QST + kst * 16 + (lane >> 4) * 8, a0, a1, a2, a3);
+#pragma unroll
+      for (int jp = 0; jp < CS / 16; ++jp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(ks + (jp * 16 + (lane & 7) + (lane >> 4) * 8) * KST + kst * 16 + ((lane >> 3) & 1) * 8, b0, b1, b2,
+                b3);
+        mma_16816(sacc[2 * jp], a0, a1, a2, a3, b0, b1);
+        mma_16816(sacc[2 * jp + 1], a0, a1, a2, a3, b2, b3);
       }
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (tg * 4 + i < Ts) sc[(tg * 4 + i) * cs + jj] = acc[i] * p.scale;
-  }
-  __syncthreads();
 
-  // warp-shuffle softmax per token row (local to this chunk); entries past C are zeroed
-  for (int t = warp; t < Ts; t += kAttnThreads / 32) {
+    // online softmax in base 2: keys past C are masked (their K rows may hold stale data)
+    float x0 = -INFINITY, x1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < CS / 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = j * 8 + 2 * t4 + (e & 1);
+        const float v = key < C ? sacc[j][e] * sl2 : -INFINITY;
+        sacc[j][e] = v;
+        if (e < 2) x0 = fmaxf(x0, v); else x1 = fmaxf(x1, v);
+      }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, o));
+      x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, o));
+    }
+    const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);   // finite: C >= 1
+    const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);
+    m0 = n0;
+    m1 = n1;
+    l0 *= al0;
+    l1 *= al1;
+    uint32_t pf[CS / 16][4];
+#pragma unroll
+    for (int j = 0; j < CS / 8; ++j) {
+      const float p0 = exp2f(sacc[j][0] - n0), p1 = exp2f(sacc[j][1] - n0);
+      const float p2 = exp2f(sacc[j][2] - n1), p3 = exp2f(sacc[j][3] - n1);
+      l0 += p0 + p1;
+      l1 += p2 + p3;
+      pf[j >> 1][(j & 1) * 2 + 0] = pack_bf16x2(p0, p1);   // row g4:   a0 (keys 16kk..), a2 (keys 16kk+8..)
+      pf[j >> 1][(j & 1) * 2 + 1] = pack_bf16x2(p2, p3);   // row g4+8: a1, a3
+    }
+#pragma unroll
+    for (int n = 0; n < HD / 8; ++n) {
+      oacc[n][0] *= al0;
+      oacc[n][1] *= al0;
+      oacc[n][2] *= al1;
+      oacc[n][3] *= al1;
+    }
+
+    // O += P V
+#pragma unroll
+    for (int kk = 0; kk < CS / 16; ++kk) {
+#pragma unroll
+      for (int np = 0; np < HD / 16; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(vs + (np * 16 + (lane & 7) + (lane >> 4) * 8) * VST + kk * 16 + ((lane >> 3) & 1) * 8, b0, b1, b2,
+                b3);
+        mma_16816(oacc[2 * np], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b0, b1);
+        mma_16816(oacc[2 * np + 1], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b2, b3);
+      }
+    }
+  }
+  cp_async_wait_all();   // a CTA left without keys (prefix shorter than planned) still drains its copies
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {   // row sums over the quad (each thread summed its own keys)
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+
+  // ---------------------------------------------------------------- push (O, max, sum) to row owners
+  const int rpo = p.rpo;
+  const int r0 = warp * 16 + g4, r1 = r0 + 8;          // block rows held by this thread
+  float* own0 = recv + ((size_t)c * rpo + (r0 % rpo)) * RST;
+  float* own1 = recv + ((size_t)c * rpo + (r1 % rpo)) * RST;
+  float* dst0 = S > 1 ? map_peer_w(own0, (uint32_t)(r0 / rpo)) : own0;
+  float* dst1 = S > 1 ? map_peer_w(own1, (uint32_t)(r1 / rpo)) : own1;
+#pragma unroll
+  for (int n = 0; n < HD / 8; ++n) {
+    const int d = n * 8 + 2 * t4;
+    *reinterpret_cast<float2*>(dst0 + d) = make_float2(oacc[n][0], oacc[n][1]);
+    *reinterpret_cast<float2*>(dst1 + d) = make_float2(oacc[n][2], oacc[n][3]);
+  }
+  if (t4 == 0) {
+    *reinterpret_cast<float2*>(dst0 + HD) = make_float2(m0, l0);
+    *reinterpret_cast<float2*>(dst1 + HD) = make_float2(m1, l1);
+  }
+  if (S > 1) {
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  } else {
+    __syncthreads();
+  }
+
+  // ---------------------------------------------------------------- merge the CTAs' partials of owned rows
+  const int rbeg = c * rpo, rend = min(kAttnRows, rbeg + rpo);
+  for (int e = tid; e < (rend - rbeg) * (HD / 4); e += kAttnThreads) {
+    const int lr = e / (HD / 4), d = (e % (HD / 4)) * 4;
+    const int row = rb * kAttnRows + rbeg + lr;         // row in this kv head's row set
+    if (row >= R) continue;
     float mx = -INFINITY;
-    for (int jj = lane; jj < C; jj += 32) mx = fmaxf(mx, sc[t * cs + jj]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
-    for (int jj = lane; jj < cs; jj += 32) {
-      const float e = jj < C ? __expf(sc[t * cs + jj] - mx) : 0.f;
-      sc[t * cs + jj] = e;
-      sum += e;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) {
-      ml[t] = mx;
-      ml[Ts + t] = sum;
-    }
-  }
-  __syncthreads();
-
-  // partial O: item = (d, group of 4 tokens); 8 keys per 16-byte load
-  for (int it = tid; it < HD * ntg; it += kAttnThreads) {
-    const int d = it % HD, tg = it / HD;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const __nv_bfloat16* vr = vs + d * VST;
-    for (int jj = 0; jj < C; jj += 8) {
-      float vf[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(vr + jj), vf);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = min(tg * 4 + i, Ts - 1);
-        const float4 p0 = *reinterpret_cast<const float4*>(sc + t * cs + jj);
-        const float4 p1 = *reinterpret_cast<const float4*>(sc + t * cs + jj + 4);
-        acc[i] = fmaf(p0.x, vf[0], acc[i]);
-        acc[i] = fmaf(p0.y, vf[1], acc[i]);
-        acc[i] = fmaf(p0.z, vf[2], acc[i]);
-        acc[i] = fmaf(p0.w, vf[3], acc[i]);
-        acc[i] = fmaf(p1.x, vf[4], acc[i]);
-        acc[i] = fmaf(p1.y, vf[5], acc[i]);
-        acc[i] = fmaf(p1.z, vf[6], acc[i]);
-        acc[i] = fmaf(p1.w, vf[7], acc[i]);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (tg * 4 + i < Ts) po[(tg * 4 + i) * HD + d] = acc[i];
-  }
-
-  // merge the S partials (fixed order) for this CTA's share of the tokens
-  if (S > 1) cluster_sync_all(); else __syncthreads();
-  const int t0 = (s * Ts) / S, t1 = ((s + 1) * Ts) / S;
-  float* wgt = ml + 2 * Ts;   // [16][Ts] merge weights
-  const uint32_t ml_local = smem_u32(ml), po_local = smem_u32(po);
-  for (int t = t0 + tid; t < t1; t += kAttnThreads) {
-    float mr[16], lr[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < S) {
-        if (S == 1) {
-          mr[r] = ml[t];
-          lr[r] = ml[Ts + t];
-        } else {
-          mr[r] = ld_dsmem_f32(mapa_shared(ml_local + t * 4u, (uint32_t)r));
-          lr[r] = ld_dsmem_f32(mapa_shared(ml_local + (Ts + t) * 4u, (uint32_t)r));
-        }
-      }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < S) mx = fmaxf(mx, mr[r]);
+    for (int s2 = 0; s2 < S; ++s2) mx = fmaxf(mx, recv[((size_t)s2 * rpo + lr) * RST + HD]);
     float den = 0.f;
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < S) {
-        mr[r] = __expf(mr[r] - mx);
-        den += mr[r] * lr[r];
-      }
-    const float inv = 1.f / den;
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < S) wgt[r * Ts + t] = mr[r] * inv;
-  }
-  __syncthreads();
-  for (int e = tid; e < (t1 - t0) * (HD / 4); e += kAttnThreads) {
-    const int t = t0 + e / (HD / 4), d = (e % (HD / 4)) * 4;
-    float4 pr[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < S) {
-        if (S == 1)
-          pr[r] = *reinterpret_cast<const float4*>(po + t * HD + d);
-        else
-          pr[r] = ld_dsmem_f32x4(mapa_shared(po_local + (uint32_t)(t * HD + d) * 4u, (uint32_t)r));
-      }
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-      if (r < S) {
-        const float w = wgt[r * Ts + t];
-        acc.x = fmaf(w, pr[r].x, acc.x);
-        acc.y = fmaf(w, pr[r].y, acc.y);
-        acc.z = fmaf(w, pr[r].z, acc.z);
-        acc.w = fmaf(w, pr[r].w, acc.w);
-      }
-    const int tok = b * Ts + t;
-    const int nt = tok / p.NT, row = tok % p.NT;
-    const int k = h * HD + d;
-    // hi / lo bf16 pair per value, 4 consecutive columns inside one 16-byte chunk
-    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    for (int s2 = 0; s2 < S; ++s2) {                    // rank order: deterministic
+      const float* src = recv + ((size_t)s2 * rpo + lr) * RST;
+      const float w = exp2f(src[HD] - mx);
+      den = fmaf(w, src[HD + 1], den);
+      const float4 o = *reinterpret_cast<const float4*>(src + d);
+      acc.x = fmaf(w, o.x, acc.x);
+      acc.y = fmaf(w, o.y, acc.y);
+      acc.z = fmaf(w, o.z, acc.z);
+      acc.w = fmaf(w, o.w, acc.w);
+    }
+    const float inv = 1.f / den;
+    const float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    const int head = kvh * rep + row / Ts, tok = b * Ts + row % Ts;
+    const int k = head * HD + d;
     __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       hi[q] = __float2bfloat16_rn(v[q]);
       lo[q] = __float2bfloat16_rn(v[q] - __bfloat162float(hi[q]));
     }
-    __nv_bfloat16* base = p.o_tiles + ((size_t)nt * p.KBo + (k >> 6)) * 2 * p.NT * 64 + sw128_elem_offset(row, k & 63);
+    __nv_bfloat16* base = p.o_tiles + operand_offset(tok, k, p.NT, p.KBo);
     *reinterpret_cast<uint2*>(base) = *reinterpret_cast<const uint2*>(hi);
     *reinterpret_cast<uint2*>(base + (size_t)p.NT * 64) = *reinterpret_cast<const uint2*>(lo);
-  }
-  // peers read this CTA's partials: exit only after every CTA has finished reading (the relaxed
-  // arrive does not wait for this CTA's global stores)
-  if (S > 1) {
-    cluster_arrive_relaxed();
-    cluster_wait();
   }
 }
 

@@ -72,7 +72,8 @@ struct GemmParams {
   int KBn;
   __nv_bfloat16* m_out;      // SWIGLU: down-GEMM operand tiles [Nt][KBm][2][NT][64]
   int KBm;
-  float* q_out;              // QKV: q [Ntok][nq][hd] fp32
+  __nv_bfloat16* q_out;      // QKV: q [B][nkv][Rpad][hd] bf16, row = head_in_group * Ts + token
+  int Rpad;                  // QKV: padded q rows per kv head (64-row attention blocks)
   __nv_bfloat16* kc;         // QKV: layer K cache [B][nkv][Lpad][hd]
   __nv_bfloat16* vct;        // QKV: layer V^T cache [B][nkv][hd][Lpad]
   const float* rope;         // QKV: [Ts][hd/2][2] (cos, sin) for positions P + j
@@ -555,11 +556,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
               r1[q] = y[2 * q + 1] * cs + y[2 * q] * sn;
             }
             if (isq) {
-              float* dst = p.q_out + ((size_t)t * p.nq + head) * p.hd;
-              *reinterpret_cast<float4*>(dst + i0) = make_float4(r0[0], r0[1], r0[2], r0[3]);
-              *reinterpret_cast<float4*>(dst + i0 + 4) = make_float4(r0[4], r0[5], r0[6], r0[7]);
-              *reinterpret_cast<float4*>(dst + i0 + half) = make_float4(r1[0], r1[1], r1[2], r1[3]);
-              *reinterpret_cast<float4*>(dst + i0 + half + 4) = make_float4(r1[4], r1[5], r1[6], r1[7]);
+              const int rep = p.nq / p.nkv;
+              __nv_bfloat16* dst =
+                  p.q_out + (((size_t)b * p.nkv + head / rep) * p.Rpad + (head % rep) * p.Ts + jt) * p.hd;
+              uint32_t a[4], c[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 x0 = __floats2bfloat162_rn(r0[2 * q], r0[2 * q + 1]);
+                __nv_bfloat162 x1 = __floats2bfloat162_rn(r1[2 * q], r1[2 * q + 1]);
+                a[q] = *reinterpret_cast<uint32_t*>(&x0);
+                c[q] = *reinterpret_cast<uint32_t*>(&x1);
+              }
+              *reinterpret_cast<uint4*>(dst + i0) = make_uint4(a[0], a[1], a[2], a[3]);
+              *reinterpret_cast<uint4*>(dst + i0 + half) = make_uint4(c[0], c[1], c[2], c[3]);
             } else {
               __nv_bfloat16* dst = p.kc + (((size_t)b * p.nkv + head) * p.Lpad + p.P + jt) * p.hd;
               uint32_t a[4], c[4];

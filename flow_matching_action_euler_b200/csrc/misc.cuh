@@ -338,4 +338,14 @@ __global__ void self_kv_kernel(const __nv_bfloat16* kc, const __nv_bfloat16* vct
   }
 }
 
+// q of the attention layout [B][nkv][Rpad][hd] (rows head_in_group * Ts + token) -> fp32 [Ntok][nq][hd]
+__global__ void q_trace_kernel(const __nv_bfloat16* qb, float* out, int B, int Ts, int nq, int nkv, int hd, int Rpad) {
+  const int n = B * Ts * nq * hd, rep = nq / nkv;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+    const int d = e % hd, head = (e / hd) % nq, t = e / (hd * nq);
+    const int b = t / Ts, j = t % Ts, g = head / rep;
+    out[e] = __bfloat162float(qb[(((size_t)b * nkv + g) * Rpad + (head % rep) * Ts + j) * hd + d]);
+  }
+}
+
 }  // namespace vla

@@ -75,8 +75,8 @@ struct vla_ae {
   int Ts = 0, Ntok = 0, NT = 0, Nt = 0, qd = 0, kd = 0, Lpad = 0;
   OpPlan op[4];
   size_t layer_wbytes = 0, layer_scales = 0;
-  int attn_S = 1, attn_cmax = 0, attn_smem = 0;
-  AttnParams attn_proto{};
+  int attn_cs = 16;           // keys per attention sub-chunk (template argument)
+  AttnParams attn_proto{};    // attention launch shape: S, span, nrb, Rpad, rpo, smem offsets
   // device memory
   std::vector<void*> allocs;
   uint8_t* wpack = nullptr;
@@ -85,8 +85,8 @@ struct vla_ae {
                 *b_out = nullptr, *w_ada = nullptr, *b_ada = nullptr, *w_fada = nullptr, *b_fada = nullptr;
   __nv_bfloat16 *kc = nullptr, *vct = nullptr, *act_x = nullptr, *act_o = nullptr, *act_m = nullptr,
                 *noise_stage = nullptr, *state_stage = nullptr;
-  float *h = nullptr, *ss = nullptr, *x = nullptr, *h_state0 = nullptr, *rope = nullptr, *out_stage = nullptr,
-        *q = nullptr;
+  __nv_bfloat16* q = nullptr;   // [B][nkv][Rpad][hd]: rows head_in_group * Ts + token, after RoPE
+  float *h = nullptr, *ss = nullptr, *x = nullptr, *h_state0 = nullptr, *rope = nullptr, *out_stage = nullptr;
   double* temb = nullptr;
   unsigned* status = nullptr;
   size_t device_bytes = 0;
@@ -154,11 +154,19 @@ GemmKernel gemm_kernel_for(OpId id, bool fp8) {
 }
 
 using AttnKernel = void (*)(const AttnParams);
-AttnKernel attn_kernel_for(int hd) {
+template <int HD>
+AttnKernel attn_kernel_cs(int cs) {
+  switch (cs) {
+    case 16: return attn_kernel<HD, 16>;
+    case 32: return attn_kernel<HD, 32>;
+    default: return attn_kernel<HD, 64>;
+  }
+}
+AttnKernel attn_kernel_for(int hd, int cs) {
   switch (hd) {
-    case 64: return attn_kernel<64>;
-    case 128: return attn_kernel<128>;
-    default: return attn_kernel<256>;
+    case 64: return attn_kernel_cs<64>(cs);
+    case 128: return attn_kernel_cs<128>(cs);
+    default: return attn_kernel_cs<256>(cs);
   }
 }
 
@@ -318,42 +326,44 @@ int validate_dims(const vla_ae_dims* d) {
 }
 
 // ------------------------------------------------------------------ attention plan
+// Clusters: one per (sample, kv head, 64-row block of the head group's rep * Ts query rows).
+// Keys are split over the cluster's CTAs in spans of a multiple of 16; the first choice fills
+// the SMs with one CTA each, fewer CTAs per cluster are tried if a cluster does not fit.
 int plan_attention(vla_ae* H, int P) {
+  const vla_ae_dims& d = H->d;
   const int L = P + H->Ts;
-  const int hd = H->d.head_dim;
-  const int groups = H->d.n_q_heads * H->d.batch;
-  int S = std::max(1, std::min({16, L, H->num_sms / std::max(1, groups)}));
-  AttnKernel kern = attn_kernel_for(hd);
-  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
-  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
-  CK(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-  // candidate cluster sizes: the preferred one, then smaller, then larger (more, shorter chunks)
-  std::vector<int> cands;
-  for (int c = S; c >= 1; --c) cands.push_back(c);
-  for (int c = S + 1; c <= std::min(16, L); ++c) cands.push_back(c);
-  for (int S0 : cands) {
-    const int cs = (int)align_up((size_t)ceil_div(L, S0), 16);   // keys per chunk, multiple of 16
-    const int S = ceil_div(L, cs);
-    const int Ts = H->Ts;
-    size_t off = (size_t)Ts * (hd + 4) * 4;   // q rows, fp32, padded by 16 bytes
+  const int hd = d.head_dim;
+  const int rep = d.n_q_heads / d.n_kv_heads;
+  const int nrb = ceil_div(rep * H->Ts, kAttnRows);
+  const int groups = nrb * d.n_kv_heads * d.batch;
+  const int S0 = std::max(1, std::min({16, L, ceil_div(H->num_sms, groups)}));
+  for (int Sc = S0; Sc >= 1; --Sc) {
+    const int span = (int)align_up((size_t)ceil_div(L, Sc), 16);
+    const int S = ceil_div(L, span);
+    const int cs = span <= 16 ? 16 : span <= 32 ? 32 : 64;
+    const int rpo = ceil_div(kAttnRows, S);
+    AttnKernel kern = attn_kernel_for(hd, cs);
+    CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+    CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
+    CK(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     AttnParams a{};
-    off = align_up(off, 16);
+    size_t off = (size_t)kAttnRows * (hd + 8) * 2;   // q rows, bf16, padded by 16 bytes
     a.off_k = (int)off;
     off = align_up(off + (size_t)cs * (hd + 8) * 2, 16);
     a.off_v = (int)off;
     off = align_up(off + (size_t)hd * (cs + 8) * 2, 16);
-    a.off_s = (int)off;
-    off = align_up(off + (size_t)Ts * cs * 4, 16);
-    a.off_o = (int)off;
-    off = align_up(off + (size_t)Ts * hd * 4, 16);
-    a.off_ml = (int)off;
-    off += (size_t)(2 + 16) * Ts * 4;
-    a.cs = cs;
+    a.off_recv = (int)off;
+    off += (size_t)S * rpo * (hd + 4) * 4;
     a.smem_bytes = (int)off;
+    a.S = S;
+    a.span = span;
+    a.nrb = nrb;
+    a.Rpad = nrb * kAttnRows;
+    a.rpo = rpo;
     if (off > (size_t)kMaxDynSmem) continue;
     if (S > 1) {
       cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(S, H->d.n_q_heads, H->d.batch);
+      cfg.gridDim = dim3(S, nrb * d.n_kv_heads, d.batch);
       cfg.blockDim = dim3(kAttnThreads);
       cfg.dynamicSmemBytes = off;
       cudaLaunchAttribute at;
@@ -370,9 +380,7 @@ int plan_attention(vla_ae* H, int P) {
       }
       if (ncl < 1) continue;
     }
-    H->attn_S = S;
-    H->attn_cmax = cs;
-    H->attn_smem = (int)off;
+    H->attn_cs = cs;
     H->attn_proto = a;
     return VLA_AE_OK;
   }
@@ -455,6 +463,7 @@ cudaError_t enqueue_op(vla_ae* H, const StepTables& T, int step, int layer, int 
       g.ss_parts = ss_in_parts;
       g.cshift = T.cq + cl * H->op[OP_QKV].Mt * 128;
       g.q_out = H->q;
+      g.Rpad = H->attn_proto.Rpad;
       g.kc = H->kc + cache;
       g.vct = H->vct + cache;
       g.rope = H->rope;
@@ -481,11 +490,9 @@ cudaError_t enqueue_op(vla_ae* H, const StepTables& T, int step, int layer, int 
       a.Ntok = H->Ntok;
       a.NT = H->NT;
       a.KBo = H->op[OP_O].KB;
-      a.S = H->attn_S;
-      a.cs = H->attn_cmax;
       a.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
-      return launch(attn_kernel_for(d.head_dim), dim3(H->attn_S, d.n_q_heads, d.batch), dim3(kAttnThreads),
-                    H->attn_smem, st, H->attn_S, true, a);
+      return launch(attn_kernel_for(d.head_dim, H->attn_cs), dim3(a.S, a.nrb * d.n_kv_heads, d.batch),
+                    dim3(kAttnThreads), a.smem_bytes, st, a.S, true, a);
     }
     case LOP_O: {  // o-projection + gated residual; writes the gate/up operand h (1 + scale_m)
       GemmParams g = gemm_common(H, OP_O, layer);
@@ -531,7 +538,8 @@ cudaError_t enqueue_layer(vla_ae* H, const StepTables& T, int step, int layer, i
   cudaError_t e;
   if ((e = enqueue_op(H, T, step, layer, LOP_QKV, ss_in_parts, st)) != cudaSuccess) return e;
   if (trace && trace->q)
-    cudaMemcpyAsync(trace->q, H->q, (size_t)H->Ntok * H->qd * 4, cudaMemcpyDeviceToDevice, st);
+    q_trace_kernel<<<64, 256, 0, st>>>(H->q, trace->q, d.batch, H->Ts, d.n_q_heads, d.n_kv_heads, d.head_dim,
+                                       H->attn_proto.Rpad);
   if (trace && trace->k && trace->v)
     self_kv_kernel<<<64, 256, 0, st>>>(H->kc + cache, H->vct + cache, trace->k, trace->v, d.batch, H->Ts,
                                        d.n_kv_heads, d.head_dim, H->n_prefix, H->Lpad);
@@ -779,7 +787,7 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   const size_t cache = L * B * d.n_kv_heads * (size_t)H->Lpad * d.head_dim;
   if ((rc = H->alloc(&H->kc, cache * 2))) return rc;
   if ((rc = H->alloc(&H->vct, cache * 2))) return rc;
-  if ((rc = H->alloc(&H->q, (size_t)H->Ntok * H->qd * 4))) return rc;
+  if ((rc = H->alloc(&H->q, B * d.n_kv_heads * (size_t)H->attn_proto.Rpad * d.head_dim * 2))) return rc;
   if ((rc = H->alloc(&H->act_x, (size_t)H->Nt * H->op[OP_QKV].KB * 2 * H->NT * 64 * 2))) return rc;
   if ((rc = H->alloc(&H->act_o, (size_t)H->Nt * H->op[OP_O].KB * 2 * H->NT * 64 * 2))) return rc;
   if ((rc = H->alloc(&H->act_m, (size_t)H->Nt * H->op[OP_D].KB * 2 * H->NT * 64 * 2))) return rc;
