@@ -17,12 +17,13 @@ __all__ = [
     "lib", "VlaAeDims", "VlaAeWeights", "VlaAeTrace", "VlaAeError", "ActionExpert",
     "vla_ae_create", "vla_ae_set_prefix", "vla_ae_denoise", "vla_ae_denoise_host", "vla_ae_status",
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
-    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
-    "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES",
+    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "BF16", "FP8_E4M3", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
+    "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES", "Q_ENGINE", "ENGINE_PER_OP", "ENGINE_PERSISTENT",
 ]
 
 BF16, FP8_E4M3 = 0, 1
-Q_KERNELS_PER_LOOP, Q_WEIGHT_BYTES, Q_KV_BYTES, Q_DEVICE_BYTES, Q_SPLITS, Q_OP_BYTES = 1, 2, 3, 4, 5, 6
+Q_KERNELS_PER_LOOP, Q_WEIGHT_BYTES, Q_KV_BYTES, Q_DEVICE_BYTES, Q_SPLITS, Q_OP_BYTES, Q_ENGINE = 1, 2, 3, 4, 5, 6, 7
+ENGINE_PER_OP, ENGINE_PERSISTENT = 0, 1
 OK, EINVAL, ENOMEM, ECUDA, ENOPREFIX, ETIMEOUT, EUNSUPPORTED = 0, -1, -2, -3, -4, -5, -6
 
 if not os.path.exists(LIB_PATH):
@@ -78,6 +79,7 @@ vla_ae_debug_velocity = _sig("vla_ae_debug_velocity", ctypes.c_int, _H, ctypes.c
 vla_ae_debug_weight = _sig("vla_ae_debug_weight", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_bench_op = _sig("vla_ae_bench_op", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P)
 vla_ae_debug_wait_probe = _sig("vla_ae_debug_wait_probe", ctypes.c_int, _H, ctypes.c_uint)
+vla_ae_set_engine = _sig("vla_ae_set_engine", ctypes.c_int, _H, ctypes.c_int)
 vla_ae_set_prefix_static = _sig("vla_ae_set_prefix_static", ctypes.c_int, _H, _P, _P, ctypes.c_int, _P, _P)
 
 
@@ -184,6 +186,14 @@ class ActionExpert:
 
     def debug_wait_probe(self, attempts: int):
         _check(vla_ae_debug_wait_probe(self.handle, int(attempts)), "vla_ae_debug_wait_probe")
+
+    def set_engine(self, engine: int):
+        """ENGINE_PER_OP or ENGINE_PERSISTENT (raises EUNSUPPORTED where the latter is unavailable)."""
+        _check(vla_ae_set_engine(self.handle, engine), "vla_ae_set_engine")
+
+    @property
+    def engine(self) -> int:
+        return self.query(Q_ENGINE)
 
     def bench_op(self, op: int, count: int, steps: int, stream=None):
         _check(vla_ae_bench_op(self.handle, op, count, steps, _stream_ptr(stream)), "vla_ae_bench_op")

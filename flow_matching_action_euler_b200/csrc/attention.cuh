@@ -37,7 +37,7 @@ struct AttnParams {
   int Rpad;                  // nrb * 64
   int rpo;                   // rows owned per CTA in the merge = ceil(64 / S)
   float scale;               // 1 / sqrt(hd)
-  int off_k, off_v, off_recv, smem_bytes;
+  int off_recv, smem_bytes;   // receive buffer after the block's staging area
 };
 
 __device__ __forceinline__ void ldsm_x4(const void* smem_row_addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -59,60 +59,60 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <int HD, int CS>
-__global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constant__ AttnParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
+// Shared-memory bytes of one 64-row block: q rows, one sub-chunk of K rows and of V^T columns.
+__host__ __device__ constexpr int attn_block_smem(int hd, int cs) {
+  return kAttnRows * (hd + 8) * 2 + cs * (hd + 8) * 2 + hd * (cs + 8) * 2;
+}
+
+// Partial attention of one 64-row block over the keys [kbeg, kend) of one (sample, kv head):
+// 4 warps x 16 rows, `tid` in [0, 128).  `sync()` is a barrier over those 128 threads;
+// `before_self()` runs between issuing the prefix copies of the first sub-chunk and the copies
+// of anything the loop writes (self K/V rows, q).  Keys past L inside the last 8-column V^T
+// copy stay inside the Lpad-long cache rows and meet P = 0; spans are multiples of 16 keys.
+// On return `row_dst(r)` (r = 0..63) holds the row's unnormalised O[HD], then (max, sum) in
+// base-2 units at [HD], [HD + 1].
+template <int HD, int CS, typename Sync, typename BeforeSelf, typename RowDst>
+__device__ __forceinline__ void attn_block_partial(uint8_t* smem, const __nv_bfloat16* qbase,
+                                                   const __nv_bfloat16* kbase, const __nv_bfloat16* vbase, int P,
+                                                   int Lpad, int kbeg, int kend, float scale, int tid, Sync sync,
+                                                   BeforeSelf before_self, RowDst row_dst) {
   constexpr int QST = HD + 8, KST = HD + 8, VST = CS + 8;   // padded rows (bf16): conflict-free ldmatrix
-  constexpr int RST = HD + 4;                                 // receive row: O[HD], max, sum
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp = tid >> 5, lane = tid & 31;
   const int g4 = lane >> 2, t4 = lane & 3;
-  const int c = blockIdx.x, rb = blockIdx.y % p.nrb, kvh = blockIdx.y / p.nrb, b = blockIdx.z;
-  const int S = p.S, Ts = p.Ts;
-  const int L = p.P + Ts;
-  const int kbeg = c * p.span, kend = min(L, kbeg + p.span);   // this CTA's keys (>= 1 of them)
-  const int nch = (kend - kbeg + CS - 1) / CS;
-  const int rep = p.nq / p.nkv, R = rep * Ts;
+  const int nch = kend > kbeg ? (kend - kbeg + CS - 1) / CS : 0;
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem);                              // [64][QST]
+  __nv_bfloat16* ks = qs + kAttnRows * QST;                                               // [CS][KST]
+  __nv_bfloat16* vs = ks + CS * KST;                                                      // [HD][VST]
 
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem);              // [64][QST]
-  __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(smem + p.off_k);    // [CS][KST]
-  __nv_bfloat16* vs = reinterpret_cast<__nv_bfloat16*>(smem + p.off_v);    // [HD][VST]
-  float* recv = reinterpret_cast<float*>(smem + p.off_recv);               // [S][rpo][RST]
-
-  pdl_trigger();
-  const __nv_bfloat16* kbase = p.kc + ((size_t)b * p.nkv + kvh) * p.Lpad * HD;
-  const __nv_bfloat16* vbase = p.vct + ((size_t)b * p.nkv + kvh) * (size_t)HD * p.Lpad;
-  // K rows and V^T columns of sub-chunk j0 (part = 0: prefix only, 1: self only, 2: all).  The
-  // spans are multiples of 16 keys, so an 8-column V^T copy never crosses into the next CTA's
-  // keys; copies past L stay inside the Lpad-long cache rows and meet P = 0.
+  // K rows and V^T columns of sub-chunk j0 (part = 0: prefix only, 1: self only, 2: all)
   auto issue_kv = [&](int j0, int part) {
     for (int e = tid; e < CS * (HD / 8); e += kAttnThreads) {
       const int jj = j0 + e / (HD / 8), cc = e % (HD / 8);
-      if (jj < kend && (part == 2 || (jj < p.P) == (part == 0)))
+      if (jj < kend && (part == 2 || (jj < P) == (part == 0)))
         cp_async16(ks + (jj - j0) * KST + cc * 8, kbase + (size_t)jj * HD + cc * 8);
     }
     for (int e = tid; e < HD * (CS / 8); e += kAttnThreads) {
       const int d = e / (CS / 8), cc = e % (CS / 8);
       const int key0 = j0 + cc * 8;
       if (key0 < kend) {
-        if (part == 2 || (key0 + 8 <= p.P) == (part == 0))
-          cp_async16(vs + d * VST + cc * 8, vbase + (size_t)d * p.Lpad + key0);
-      } else if (part != 1) {   // zero columns past the CTA's keys: P is 0 there, V must be finite
+        if (part == 2 || (key0 + 8 <= P) == (part == 0))
+          cp_async16(vs + d * VST + cc * 8, vbase + (size_t)d * Lpad + key0);
+      } else if (part != 1) {   // zero columns past the keys: P is 0 there, V must be finite
         *reinterpret_cast<uint4*>(vs + d * VST + cc * 8) = make_uint4(0, 0, 0, 0);
       }
     }
   };
   issue_kv(kbeg, 0);
   cp_async_commit();
-  pdl_wait();
+  before_self();
   issue_kv(kbeg, 1);
-  const __nv_bfloat16* qbase = p.q + (((size_t)b * p.nkv + kvh) * p.Rpad + (size_t)rb * kAttnRows) * HD;
   for (int e = tid; e < kAttnRows * (HD / 8); e += kAttnThreads) {
     const int r = e / (HD / 8), cc = e % (HD / 8);
     cp_async16(qs + r * QST + cc * 8, qbase + (size_t)r * HD + cc * 8);
   }
   cp_async_commit();
 
-  const float sl2 = p.scale * 1.4426950408889634f;   // 1/sqrt(hd) * log2(e)
+  const float sl2 = scale * 1.4426950408889634f;   // 1/sqrt(hd) * log2(e)
   const int arow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows g4 and g4 + 8 of the warp
   float oacc[HD / 8][4];
@@ -122,12 +122,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
   for (int ch = 0; ch < nch; ++ch) {
     const int j0 = kbeg + ch * CS, C = min(CS, kend - j0);
     if (ch > 0) {
-      __syncthreads();   // every warp is done with the previous sub-chunk
+      sync();   // every warp is done with the previous sub-chunk
       issue_kv(j0, 2);
       cp_async_commit();
     }
     cp_async_wait_all();
-    __syncthreads();
+    sync();
 
     // S = Q K^T for the warp's 16 rows
     float sacc[CS / 8][4];
@@ -200,20 +200,15 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
       }
     }
   }
-  cp_async_wait_all();   // a CTA left without keys (prefix shorter than planned) still drains its copies
+  cp_async_wait_all();   // a block left without keys (prefix shorter than planned) still drains its copies
 #pragma unroll
   for (int o = 1; o <= 2; o <<= 1) {   // row sums over the quad (each thread summed its own keys)
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
-
-  // ---------------------------------------------------------------- push (O, max, sum) to row owners
-  const int rpo = p.rpo;
-  const int r0 = warp * 16 + g4, r1 = r0 + 8;          // block rows held by this thread
-  float* own0 = recv + ((size_t)c * rpo + (r0 % rpo)) * RST;
-  float* own1 = recv + ((size_t)c * rpo + (r1 % rpo)) * RST;
-  float* dst0 = S > 1 ? map_peer_w(own0, (uint32_t)(r0 / rpo)) : own0;
-  float* dst1 = S > 1 ? map_peer_w(own1, (uint32_t)(r1 / rpo)) : own1;
+  const int r0 = warp * 16 + g4, r1 = r0 + 8;
+  float* dst0 = row_dst(r0);
+  float* dst1 = row_dst(r1);
 #pragma unroll
   for (int n = 0; n < HD / 8; ++n) {
     const int d = n * 8 + 2 * t4;
@@ -224,28 +219,32 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
     *reinterpret_cast<float2*>(dst0 + HD) = make_float2(m0, l0);
     *reinterpret_cast<float2*>(dst1 + HD) = make_float2(m1, l1);
   }
-  if (S > 1) {
-    cluster_arrive_release();
-    cluster_wait_acquire();
-  } else {
-    __syncthreads();
-  }
+}
 
-  // ---------------------------------------------------------------- merge the CTAs' partials of owned rows
-  const int rbeg = c * rpo, rend = min(kAttnRows, rbeg + rpo);
-  for (int e = tid; e < (rend - rbeg) * (HD / 4); e += kAttnThreads) {
-    const int lr = e / (HD / 4), d = (e % (HD / 4)) * 4;
-    const int row = rb * kAttnRows + rbeg + lr;         // row in this kv head's row set
+// Merge of the S partials (rank order: deterministic) of rows [rbeg, rend) of a 64-row block and
+// write of the o-projection's hi/lo operand.  `src(s, r)` points at partial s of block row r
+// (O[HD], max, sum); GLOBAL partials written by other SMs are read through L2.
+template <int HD, bool GLOBAL, typename Src>
+__device__ __forceinline__ void attn_merge_rows(Src src, int S, int rbeg, int rend, int row_base, int R, int Ts,
+                                                int b, int kvh, int rep, __nv_bfloat16* o_tiles, int NT, int KBo,
+                                                int tid, int nthreads) {
+  auto ld1 = [](const float* a) { return GLOBAL ? __ldcg(a) : *a; };
+  auto ld4 = [](const float* a) {
+    return GLOBAL ? __ldcg(reinterpret_cast<const float4*>(a)) : *reinterpret_cast<const float4*>(a);
+  };
+  for (int e = tid; e < (rend - rbeg) * (HD / 4); e += nthreads) {
+    const int r = rbeg + e / (HD / 4), d = (e % (HD / 4)) * 4;
+    const int row = row_base + r;                       // row in this kv head's row set
     if (row >= R) continue;
     float mx = -INFINITY;
-    for (int s2 = 0; s2 < S; ++s2) mx = fmaxf(mx, recv[((size_t)s2 * rpo + lr) * RST + HD]);
+    for (int s2 = 0; s2 < S; ++s2) mx = fmaxf(mx, ld1(src(s2, r) + HD));
     float den = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s2 = 0; s2 < S; ++s2) {                    // rank order: deterministic
-      const float* src = recv + ((size_t)s2 * rpo + lr) * RST;
-      const float w = exp2f(src[HD] - mx);
-      den = fmaf(w, src[HD + 1], den);
-      const float4 o = *reinterpret_cast<const float4*>(src + d);
+    for (int s2 = 0; s2 < S; ++s2) {
+      const float* sp = src(s2, r);
+      const float w = exp2f(ld1(sp + HD) - mx);
+      den = fmaf(w, ld1(sp + HD + 1), den);
+      const float4 o = ld4(sp + d);
       acc.x = fmaf(w, o.x, acc.x);
       acc.y = fmaf(w, o.y, acc.y);
       acc.z = fmaf(w, o.z, acc.z);
@@ -261,10 +260,45 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
       hi[q] = __float2bfloat16_rn(v[q]);
       lo[q] = __float2bfloat16_rn(v[q] - __bfloat162float(hi[q]));
     }
-    __nv_bfloat16* base = p.o_tiles + operand_offset(tok, k, p.NT, p.KBo);
+    __nv_bfloat16* base = o_tiles + operand_offset(tok, k, NT, KBo);
     *reinterpret_cast<uint2*>(base) = *reinterpret_cast<const uint2*>(hi);
-    *reinterpret_cast<uint2*>(base + (size_t)p.NT * 64) = *reinterpret_cast<const uint2*>(lo);
+    *reinterpret_cast<uint2*>(base + (size_t)NT * 64) = *reinterpret_cast<const uint2*>(lo);
   }
+}
+
+template <int HD, int CS>
+__global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int RST = HD + 4;                                 // receive row: O[HD], max, sum
+  const int tid = threadIdx.x;
+  const int c = blockIdx.x, rb = blockIdx.y % p.nrb, kvh = blockIdx.y / p.nrb, b = blockIdx.z;
+  const int S = p.S;
+  const int L = p.P + p.Ts;
+  const int kbeg = c * p.span, kend = min(L, kbeg + p.span);
+  const int rep = p.nq / p.nkv;
+  float* recv = reinterpret_cast<float*>(smem + p.off_recv);   // [S][rpo][RST]
+  const int rpo = p.rpo;
+
+  pdl_trigger();
+  const size_t cache = (size_t)b * p.nkv + kvh;
+  attn_block_partial<HD, CS>(
+      smem, p.q + (cache * p.Rpad + (size_t)rb * kAttnRows) * HD, p.kc + cache * p.Lpad * HD,
+      p.vct + cache * HD * p.Lpad, p.P, p.Lpad, kbeg, kend, p.scale, tid, [] { __syncthreads(); },
+      [] { pdl_wait(); },
+      [&](int r) {   // push to the row's owner rank
+        float* own = recv + ((size_t)c * rpo + (r % rpo)) * RST;
+        return S > 1 ? map_peer_w(own, (uint32_t)(r / rpo)) : own;
+      });
+  if (S > 1) {
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  } else {
+    __syncthreads();
+  }
+  const int rbeg = c * rpo, rend = min(kAttnRows, rbeg + rpo);
+  attn_merge_rows<HD, false>([&](int s2, int r) { return recv + ((size_t)s2 * rpo + (r - rbeg)) * RST; }, S, rbeg,
+                             rend, rb * kAttnRows, rep * p.Ts, p.Ts, b, kvh, rep, p.o_tiles, p.NT, p.KBo, tid,
+                             kAttnThreads);
 }
 
 }  // namespace vla

@@ -24,6 +24,7 @@
 #include "ptx.cuh"
 #include "gemm.cuh"
 #include "attention.cuh"
+#include "loop.cuh"
 #include "misc.cuh"
 
 using namespace vla;
@@ -62,8 +63,10 @@ struct StepTables {
   float* fmod = nullptr;   // [steps][2H]
   float* cq = nullptr;     // [steps][L][Mt_qkv * 128]: W_qkv . shift_attn
   float* cg = nullptr;     // [steps][L][Mt_gu * 128]:  W_gu . shift_mlp
+  unsigned* ctr = nullptr;  // persistent engine: per-step counter blocks [steps][ctr_step]
   cudaGraphExec_t exec = nullptr;
   int captured_prefix = -1;
+  int captured_engine = -1;
 };
 
 }  // namespace
@@ -77,6 +80,13 @@ struct vla_ae {
   size_t layer_wbytes = 0, layer_scales = 0;
   int attn_cs = 16;           // keys per attention sub-chunk (template argument)
   AttnParams attn_proto{};    // attention launch shape: S, span, nrb, Rpad, rpo, smem offsets
+  // persistent engine
+  bool loop_ok = false;       // planned (bf16, one n-tile, units fit the SMs)
+  bool use_loop = false;      // selected
+  int loop_cs = 16;           // attention sub-chunk of the persistent kernel
+  LoopParams loop_proto{};    // plan: op shapes, smem layout, task lists, scratch
+  size_t ctr_step = 0;        // counters per launch (layers x ctr_layer + abort word)
+  unsigned* loop_dbg_ctr = nullptr;   // counter block of debug launches
   // device memory
   std::vector<void*> allocs;
   uint8_t* wpack = nullptr;
@@ -140,6 +150,23 @@ cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
   }
   cfg.attrs = attrs;
   cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, arg);
+}
+
+// One CTA per SM for the whole launch: the cooperative attribute makes the launch fail instead of
+// leaving CTAs unscheduled while others wait for them.
+template <typename Kern, typename Arg>
+cudaError_t launch_coop(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, const Arg& arg) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeCooperative;
+  at.val.cooperative = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, arg);
 }
 
@@ -347,11 +374,7 @@ int plan_attention(vla_ae* H, int P) {
     CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
     CK(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     AttnParams a{};
-    size_t off = (size_t)kAttnRows * (hd + 8) * 2;   // q rows, bf16, padded by 16 bytes
-    a.off_k = (int)off;
-    off = align_up(off + (size_t)cs * (hd + 8) * 2, 16);
-    a.off_v = (int)off;
-    off = align_up(off + (size_t)hd * (cs + 8) * 2, 16);
+    size_t off = (size_t)attn_block_smem(hd, cs);   // q rows, K rows, V^T columns (bf16, padded rows)
     a.off_recv = (int)off;
     off += (size_t)S * rpo * (hd + 4) * 4;
     a.smem_bytes = (int)off;
@@ -385,6 +408,189 @@ int plan_attention(vla_ae* H, int P) {
     return VLA_AE_OK;
   }
   return VLA_AE_EUNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ persistent engine plan
+using LoopKernel = void (*)(const LoopParams);
+template <int HD>
+LoopKernel loop_kernel_cs(int cs) {
+  return cs <= 16 ? loop_kernel<HD, 16> : loop_kernel<HD, 32>;
+}
+LoopKernel loop_kernel_for(int hd, int cs) {
+  switch (hd) {
+    case 64: return loop_kernel_cs<64>(cs);
+    case 128: return loop_kernel_cs<128>(cs);
+    default: return loop_kernel_cs<256>(cs);
+  }
+}
+
+// Work units and shared-memory layout of the persistent kernel.  Per GEMM: m-tiles per unit and
+// split-K chosen so that every unit fits one SM (units <= SMs), the largest unit streams the
+// fewest weight tiles, and its activation slice fits the operand buffer.  Attention: one unit
+// per (sample, kv head, 64-row block, key span), spans planned for the longest prefix (a shorter
+// prefix leaves trailing spans empty, which the merge weighs by zero).  Units are dealt to the
+// CTAs round-robin, phase after phase, so each phase is spread over all SMs.  Leaves
+// H->loop_ok false when the shape is outside the engine (fp8, more than one n-tile, ...).
+int plan_loop(vla_ae* H) {
+  const vla_ae_dims& d = H->d;
+  H->loop_ok = false;
+  if (H->fp8 || H->Nt != 1 || H->NT > 128) return VLA_AE_OK;
+  const int G = H->num_sms, NT = H->NT, hd = d.head_dim;
+  LoopParams lp{};
+  const OpId ids[4] = {OP_QKV, OP_O, OP_GU, OP_D};
+  // attention units
+  const int rep = d.n_q_heads / d.n_kv_heads;
+  const int nrb = ceil_div(rep * H->Ts, kAttnRows);
+  const int groups = nrb * d.n_kv_heads * d.batch;
+  const int Lmax = d.max_prefix + H->Ts;
+  // key spans: up to 8 per block (one round of loads per merged value), as many as the SMs allow
+  const int S0 = std::max(1, std::min({Lmax, 8, G / groups}));
+  const int span = (int)align_up((size_t)ceil_div(Lmax, S0), 16);
+  const int attn_S = ceil_div(Lmax, span);
+  const int cs = span <= 16 ? 16 : 32;
+  const size_t attn_bytes = (size_t)attn_block_smem(hd, cs);
+  // GEMM units.  Latency model of one phase on the busiest CTA (microseconds, measured on the
+  // persistent kernel): 1.5 per unit (accumulator hand-off, split wait, epilogue), 0.3 per
+  // 128-row accumulator (partial store and reduction), 0.12 per weight tile already in the ring
+  // (MMA issue), 0.36 per tile that must still stream when the phase starts (phase load above
+  // the ring depth).  Search over operand-slice caps, which trade ring depth against split count.
+  double best_cost = 1e30;
+  int best_cfg[4][2] = {};
+  for (size_t cap = 16 * 1024; cap <= 96 * 1024; cap += 8 * 1024) {
+    int cfg[4][2], load[4], mpc_max = 1;
+    double cost = 0.0;
+    size_t slice_used = 0;
+    bool ok = true;
+    for (int i = 0; i < 4 && ok; ++i) {
+      const OpPlan& q = H->op[ids[i]];
+      double best = 1e30;
+      cfg[i][0] = 0;
+      for (int mpc : {1, 2, 4}) {
+        if (mpc * 2 * NT > 256 || (mpc > 1 && mpc > q.Mt)) continue;
+        const int ng = ceil_div(q.Mt, mpc);
+        for (int S = 1; S <= q.KBt && ng * S <= 4 * G; ++S) {
+          const int nk = ceil_div(q.KBt, S);
+          if ((size_t)nk * 2 * NT * 128 > cap) continue;
+          const int per_cta = ceil_div(ng * S, G);
+          const double c = 0.12 * per_cta * std::min(mpc, q.Mt) * nk + 0.3 * per_cta * std::min(mpc, q.Mt) + 1.5 * per_cta;
+          if (c < best - 1e-9) {
+            best = c;
+            cfg[i][0] = mpc;
+            cfg[i][1] = S;
+            load[i] = per_cta * std::min(mpc, q.Mt) * nk;
+          }
+        }
+      }
+      if (!cfg[i][0]) ok = false;
+      if (!ok) break;
+      mpc_max = std::max(mpc_max, cfg[i][0]);
+      cost += best;
+      slice_used = std::max(slice_used, (size_t)ceil_div(q.KBt, cfg[i][1]) * 2 * NT * 128);
+    }
+    if (!ok) continue;
+    const size_t op_bytes = align_up(std::max(slice_used, attn_bytes), 1024);
+    const size_t fixed = op_bytes + align_up((size_t)(kMathThreads + NT + NT * 32 * mpc_max) * 4, 16);
+    const long long avail = (long long)kMaxDynSmem - 1024 - (long long)fixed - 1024;
+    const int stages = (int)std::min<long long>(24, std::max<long long>(0, avail / kTileBytes));
+    if (stages < 2) continue;
+    for (int i = 0; i < 4; ++i) cost += 0.36 * std::max(0, load[i] - stages);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      std::memcpy(best_cfg, cfg, sizeof(cfg));
+    }
+  }
+  if (best_cost >= 1e30) return VLA_AE_OK;
+  int ctr = kPhases, mpc_max = 1, units_max = 1;
+  size_t slice_used = 0;
+  for (int i = 0; i < 4; ++i) {
+    const OpPlan& q = H->op[ids[i]];
+    LoopOp& o = lp.op[i];
+    o.Mt = q.Mt;
+    o.mpc = best_cfg[i][0];
+    o.KBt = q.KBt;
+    o.KB = q.KB;
+    o.S = best_cfg[i][1];
+    o.O = q.O;
+    o.ngroups = ceil_div(q.Mt, o.mpc);
+    o.parts_out = o.ngroups * o.S;
+    o.ctr_base = ctr;
+    o.woff = q.woff;
+    ctr += o.ngroups;
+    mpc_max = std::max(mpc_max, o.mpc);
+    units_max = std::max(units_max, o.ngroups * o.S);
+    slice_used = std::max(slice_used, (size_t)ceil_div(q.KBt, o.S) * 2 * NT * 128);
+  }
+  lp.attn_S = attn_S;
+  lp.attn_span = span;
+  lp.nrb = nrb;
+  lp.attn_ctr_base = ctr;
+  ctr += groups;
+  lp.ctr_layer = (int)align_up((size_t)ctr, 32);
+  // task lists
+  std::vector<std::vector<uint32_t>> per(G);
+  int cursor = 0;
+  for (int ph = 0; ph < kPhases; ++ph) {
+    const int units = ph == PH_ATTN ? groups * attn_S : lp.op[loop_phase_op(ph)].ngroups * lp.op[loop_phase_op(ph)].S;
+    std::vector<char> has(G, 0);
+    for (int u = 0; u < units; ++u, ++cursor) {
+      per[cursor % G].push_back((uint32_t)ph << 24 | (uint32_t)u);
+      has[cursor % G] = 1;
+    }
+    lp.phase_target[ph] = (int)std::count(has.begin(), has.end(), 1);
+  }
+  std::vector<uint32_t> tasks((size_t)G * kLoopMaxTasks, 0);
+  std::vector<int> ntasks(G, 0);
+  for (int c = 0; c < G; ++c) {
+    if ((int)per[c].size() > kLoopMaxTasks) return VLA_AE_OK;
+    ntasks[c] = (int)per[c].size();
+    std::copy(per[c].begin(), per[c].end(), tasks.begin() + (size_t)c * kLoopMaxTasks);
+  }
+  // shared memory: ring | operand slice (or attention staging) | misc | barriers
+  const size_t op_bytes = align_up(std::max(slice_used, attn_bytes), 1024);
+  const size_t misc = (size_t)(kMathThreads + NT + NT * 32 * mpc_max) * 4;
+  const size_t fixed = op_bytes + align_up(misc, 16);
+  const size_t avail = (size_t)kMaxDynSmem - 1024 - fixed - 1024;
+  const int stages = (int)std::min<size_t>(24, avail / kTileBytes);
+  if (stages < 2) return VLA_AE_OK;
+  size_t off = (size_t)stages * kTileBytes;
+  lp.off_op = (int)off;
+  off += op_bytes;
+  lp.off_misc = (int)off;
+  off += align_up(misc, 16);
+  lp.off_bar = (int)off;
+  off += (size_t)(2 * stages + 8) * 8 + 4 + kLoopMaxTasks * 4;
+  lp.smem_bytes = (int)(off + 1024);
+  lp.stages = stages;
+  lp.mpc_max = mpc_max;
+  lp.acc_cols = mpc_max * 2 * NT;
+  lp.tmem_cols = 2 * lp.acc_cols <= 32 ? 32 : 2 * lp.acc_cols <= 64 ? 64 : 2 * lp.acc_cols <= 128 ? 128 : 2 * lp.acc_cols <= 256 ? 256 : 512;
+  if (2 * lp.acc_cols > 512 || lp.smem_bytes > kMaxDynSmem) return VLA_AE_OK;
+  LoopKernel kern = loop_kernel_for(hd, cs);
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lp.smem_bytes));
+  CK(cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+  int per_sm = 0;
+  CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLoopThreads, lp.smem_bytes));
+  if (per_sm < 1) return VLA_AE_OK;
+  // device buffers (fixed for the handle's lifetime)
+  lp.gpart_unit = (size_t)128 * mpc_max * NT;
+  int rc;
+  if ((rc = H->alloc(&lp.gpart, (size_t)units_max * lp.gpart_unit * 4))) return rc;
+  if ((rc = H->alloc(&lp.apart, (size_t)groups * attn_S * kAttnRows * (hd + 4) * 4))) return rc;
+  uint32_t* dtasks = nullptr;
+  int* dntasks = nullptr;
+  if ((rc = H->alloc(&dtasks, tasks.size() * 4))) return rc;
+  if ((rc = H->alloc(&dntasks, (size_t)G * 4))) return rc;
+  CK(cudaMemcpy(dtasks, tasks.data(), tasks.size() * 4, cudaMemcpyHostToDevice));
+  CK(cudaMemcpy(dntasks, ntasks.data(), (size_t)G * 4, cudaMemcpyHostToDevice));
+  lp.tasks = dtasks;
+  lp.ntasks = dntasks;
+  H->ctr_step = (size_t)d.n_layers * lp.ctr_layer + 32;
+  if ((rc = H->alloc(&H->loop_dbg_ctr, H->ctr_step * 4))) return rc;
+  H->loop_cs = cs;
+  H->loop_proto = lp;
+  H->loop_ok = true;
+  H->use_loop = true;
+  return VLA_AE_OK;
 }
 
 // ------------------------------------------------------------------ per-op launch
@@ -583,8 +789,83 @@ cudaError_t launch_tail(const vla_ae* H, const TailParams& t, cudaStream_t st) {
 }
 
 // The whole N-step loop (what the graph holds).
+// sums-of-squares parts the last layer's down GEMM leaves for the tail kernel
+int ss_parts_final(const vla_ae* H) { return H->use_loop ? H->loop_proto.op[3].parts_out : ss_parts_of(H, OP_D); }
+
+// Persistent-engine launch over phases [(l0, ph0), (l1 - 1, ph1)) of step `step`; `ctr` is a
+// zeroed counter block of ctr_step words.
+cudaError_t launch_loop(const vla_ae* H, const StepTables& T, int step, unsigned* ctr, int l0, int ph0, int l1,
+                        int ph1, int ss_first, cudaStream_t st) {
+  const vla_ae_dims& d = H->d;
+  LoopParams lp = H->loop_proto;
+  lp.wpack = H->wpack;
+  lp.layer_wbytes = H->layer_wbytes;
+  lp.l0 = l0;
+  lp.ph0 = ph0;
+  lp.l1 = l1;
+  lp.ph1 = ph1;
+  lp.L = d.n_layers;
+  lp.Ntok = H->Ntok;
+  lp.NT = H->NT;
+  lp.act_x = H->act_x;
+  lp.act_o = H->act_o;
+  lp.act_m = H->act_m;
+  lp.h = H->h;
+  lp.ss = H->ss;
+  lp.ss_parts_first = ss_first;
+  lp.q = H->q;
+  lp.Rpad = H->attn_proto.Rpad;
+  lp.kc = H->kc;
+  lp.vct = H->vct;
+  lp.cache_layer = (size_t)d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+  lp.rope = H->rope;
+  lp.nq = d.n_q_heads;
+  lp.nkv = d.n_kv_heads;
+  lp.hd = d.head_dim;
+  lp.Ts = H->Ts;
+  lp.P = H->n_prefix;
+  lp.Lpad = H->Lpad;
+  lp.B = d.batch;
+  lp.cq_stride = H->op[OP_QKV].Mt * 128;
+  lp.cg_stride = H->op[OP_GU].Mt * 128;
+  lp.mod = T.mod + (size_t)step * d.n_layers * 6 * d.hidden;
+  lp.cq = T.cq + (size_t)step * d.n_layers * lp.cq_stride;
+  lp.cg = T.cg + (size_t)step * d.n_layers * lp.cg_stride;
+  lp.inv_h = 1.0f / (float)d.hidden;
+  lp.eps = d.rms_eps;
+  lp.H = d.hidden;
+  lp.scale = (float)(1.0 / std::sqrt((double)d.head_dim));
+  lp.ctr = ctr;
+  lp.status = H->status;
+  return launch_coop(loop_kernel_for(d.head_dim, H->loop_cs), dim3(H->num_sms), dim3(kLoopThreads), lp.smem_bytes,
+                     st, lp);
+}
+
 cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
   const int N = T.steps, L = H->d.n_layers;
+  if (H->use_loop) {
+    cudaError_t e = cudaMemsetAsync(T.ctr, 0, (size_t)N * H->ctr_step * 4, st);
+    if (e != cudaSuccess) return e;
+    TailParams t0 = tail_common(H);
+    t0.init_from_noise = 1;
+    t0.do_in = 1;
+    t0.sc_next = layer_mod(H, T, 0, 0).scale_a;
+    if ((e = launch_tail(H, t0, st)) != cudaSuccess) return e;
+    for (int k = 0; k < N; ++k) {
+      if ((e = launch_loop(H, T, k, T.ctr + (size_t)k * H->ctr_step, 0, 0, L, kPhases, 1, st)) != cudaSuccess) return e;
+      TailParams t = tail_common(H);
+      t.ss_parts = ss_parts_final(H);
+      t.shift_f = T.fmod + (size_t)k * 2 * H->d.hidden;
+      t.scale_f = t.shift_f + H->d.hidden;
+      t.dt = -1.0f / (float)N;
+      t.do_out = 1;
+      t.do_in = k + 1 < N;
+      if (t.do_in) t.sc_next = layer_mod(H, T, k + 1, 0).scale_a;
+      t.out = k + 1 == N ? H->out_stage : nullptr;
+      if ((e = launch_tail(H, t, st)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   TailParams t0 = tail_common(H);
   t0.init_from_noise = 1;
   t0.do_in = 1;
@@ -640,6 +921,7 @@ int get_tables(vla_ae* H, int steps, StepTables** out) {
   const size_t rq = (size_t)H->op[OP_QKV].Mt * 128, rg = (size_t)H->op[OP_GU].Mt * 128;
   if ((rc = H->alloc(&T.cq, (size_t)steps * d.n_layers * rq * 4))) return rc;
   if ((rc = H->alloc(&T.cg, (size_t)steps * d.n_layers * rg * 4))) return rc;
+  if (H->loop_ok && (rc = H->alloc(&T.ctr, (size_t)steps * H->ctr_step * 4))) return rc;
   for (int l = 0; l < d.n_layers; ++l) {
     const uint8_t* wl = H->wpack + (size_t)l * H->layer_wbytes;
     const float* sl = H->fp8 ? H->wscale + (size_t)l * H->layer_scales : nullptr;
@@ -663,7 +945,7 @@ int get_tables(vla_ae* H, int steps, StepTables** out) {
 }
 
 int ensure_graph(vla_ae* H, StepTables* T) {
-  if (T->exec && T->captured_prefix == H->n_prefix) return VLA_AE_OK;
+  if (T->exec && T->captured_prefix == H->n_prefix && T->captured_engine == (int)H->use_loop) return VLA_AE_OK;
   if (T->exec) {
     cudaGraphExecDestroy(T->exec);
     T->exec = nullptr;
@@ -681,6 +963,7 @@ int ensure_graph(vla_ae* H, StepTables* T) {
   CK(cudaGraphInstantiate(&T->exec, g, 0));
   cudaGraphDestroy(g);
   T->captured_prefix = H->n_prefix;
+  T->captured_engine = (int)H->use_loop;
   return VLA_AE_OK;
 }
 
@@ -779,6 +1062,7 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   H->layer_wbytes = woff;
   H->layer_scales = soff;
   if ((rc = plan_attention(H, d.max_prefix))) return rc;
+  if ((rc = plan_loop(H))) return rc;
 
   const size_t L = d.n_layers, Hd = d.hidden, A = d.action_dim, B = d.batch;
   if ((rc = H->alloc(&H->wpack, L * H->layer_wbytes))) return rc;
@@ -794,7 +1078,8 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   if ((rc = H->alloc(&H->noise_stage, B * d.n_action_tokens * A * 2))) return rc;
   if ((rc = H->alloc(&H->state_stage, B * A * 2))) return rc;
   if ((rc = H->alloc(&H->h, (size_t)H->Ntok * Hd * 4))) return rc;
-  const int parts = std::max({1, ss_parts_of(H, OP_O), ss_parts_of(H, OP_D)});
+  int parts = std::max({1, ss_parts_of(H, OP_O), ss_parts_of(H, OP_D)});
+  if (H->loop_ok) parts = std::max({parts, H->loop_proto.op[1].parts_out, H->loop_proto.op[3].parts_out});
   if ((rc = H->alloc(&H->ss, (size_t)parts * H->Ntok * 4))) return rc;
   if ((rc = H->alloc(&H->x, B * d.n_action_tokens * A * 4))) return rc;
   if ((rc = H->alloc(&H->out_stage, B * d.n_action_tokens * A * 4))) return rc;
@@ -951,7 +1236,10 @@ int vla_ae_query(vla_ae_t H, int what, int arg, long long* value) {
   switch (what) {
     case VLA_AE_Q_KERNELS_PER_LOOP:
       if (arg < 1) return VLA_AE_EINVAL;
-      *value = 1 + (long long)arg * (5LL * d.n_layers + 1);
+      *value = 1 + (long long)arg * (H->use_loop ? 2LL : 5LL * d.n_layers + 1);
+      return VLA_AE_OK;
+    case VLA_AE_Q_ENGINE:
+      *value = H->use_loop ? VLA_AE_ENGINE_PERSISTENT : VLA_AE_ENGINE_PER_OP;
       return VLA_AE_OK;
     case VLA_AE_Q_WEIGHT_BYTES: {
       long long b = 0;
@@ -998,6 +1286,13 @@ int vla_ae_bench_op(vla_ae_t H, int op, int count, int steps, void* stream) {
   return VLA_AE_OK;
 }
 
+int vla_ae_set_engine(vla_ae_t H, int engine) {
+  if (!H || (engine != VLA_AE_ENGINE_PER_OP && engine != VLA_AE_ENGINE_PERSISTENT)) return VLA_AE_EINVAL;
+  if (engine == VLA_AE_ENGINE_PERSISTENT && !H->loop_ok) return VLA_AE_EUNSUPPORTED;
+  H->use_loop = engine == VLA_AE_ENGINE_PERSISTENT;   // graphs re-capture on their next use
+  return VLA_AE_OK;
+}
+
 int vla_ae_debug_wait_probe(vla_ae_t H, unsigned attempts) {
   if (!H || attempts == 0 || attempts > (1u << 20)) return VLA_AE_EINVAL;
   wait_probe_kernel<<<1, 32, 0, H->cap>>>(attempts, H->status);
@@ -1021,7 +1316,31 @@ int vla_ae_debug_layer(vla_ae_t H, int layer, int step, int steps, const float* 
   row_operand_kernel<<<H->Ntok, 256, 0, st>>>(H->h, H->ss, H->act_x, layer_mod(H, *T, step, layer).scale_a,
                                               H->d.hidden, H->NT, H->op[OP_QKV].KB);
   CK(cudaGetLastError());
-  CK(enqueue_layer(H, *T, step, layer, 1, st, trace));
+  if (H->use_loop) {
+    // persistent engine: the layer in one launch, or in two (through the o-projection, then the
+    // MLP) when intermediates are traced
+    const vla_ae_dims& d = H->d;
+    const size_t cache = (size_t)layer * d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+    const bool split = trace != nullptr;
+    CK(cudaMemsetAsync(H->loop_dbg_ctr, 0, H->ctr_step * 4, st));
+    CK(launch_loop(H, *T, step, H->loop_dbg_ctr, layer, 0, layer + 1, split ? (int)PH_GU : (int)kPhases, 1, st));
+    if (split) {
+      if (trace->q)
+        q_trace_kernel<<<64, 256, 0, st>>>(H->q, trace->q, d.batch, H->Ts, d.n_q_heads, d.n_kv_heads, d.head_dim,
+                                           H->attn_proto.Rpad);
+      if (trace->k && trace->v)
+        self_kv_kernel<<<64, 256, 0, st>>>(H->kc + cache, H->vct + cache, trace->k, trace->v, d.batch, H->Ts,
+                                           d.n_kv_heads, d.head_dim, H->n_prefix, H->Lpad);
+      if (trace->o) untile_kernel<<<64, 256, 0, st>>>(H->act_o, trace->o, H->Ntok, H->qd, H->NT, H->op[OP_O].KB);
+      if (trace->h_attn) CK(cudaMemcpyAsync(trace->h_attn, H->h, nh * 4, cudaMemcpyDeviceToDevice, st));
+      CK(cudaMemsetAsync(H->loop_dbg_ctr, 0, H->ctr_step * 4, st));
+      CK(launch_loop(H, *T, step, H->loop_dbg_ctr, layer, PH_GU, layer + 1, kPhases, 1, st));
+      if (trace->m) untile_kernel<<<64, 256, 0, st>>>(H->act_m, trace->m, H->Ntok, d.inter, H->NT, H->op[OP_D].KB);
+    }
+    CK(cudaGetLastError());
+  } else {
+    CK(enqueue_layer(H, *T, step, layer, 1, st, trace));
+  }
   CK(cudaMemcpyAsync(h_out, H->h, nh * 4, cudaMemcpyDeviceToDevice, st));
   CK(cudaStreamSynchronize(st));
   return VLA_AE_OK;
@@ -1041,9 +1360,15 @@ int vla_ae_debug_velocity(vla_ae_t H, int step, int steps, const float* x, float
   t0.do_in = 1;
   t0.sc_next = layer_mod(H, *T, step, 0).scale_a;
   CK(launch_tail(H, t0, st));
-  for (int l = 0; l < d.n_layers; ++l) CK(enqueue_layer(H, *T, step, l, l == 0 ? 1 : ss_parts_of(H, OP_D), st, nullptr));
+  if (H->use_loop) {
+    CK(cudaMemsetAsync(H->loop_dbg_ctr, 0, H->ctr_step * 4, st));
+    CK(launch_loop(H, *T, step, H->loop_dbg_ctr, 0, 0, d.n_layers, kPhases, 1, st));
+  } else {
+    for (int l = 0; l < d.n_layers; ++l)
+      CK(enqueue_layer(H, *T, step, l, l == 0 ? 1 : ss_parts_of(H, OP_D), st, nullptr));
+  }
   TailParams t = tail_common(H);
-  t.ss_parts = ss_parts_of(H, OP_D);
+  t.ss_parts = ss_parts_final(H);
   t.shift_f = T->fmod + (size_t)step * 2 * d.hidden;
   t.scale_f = t.shift_f + d.hidden;
   t.dt = 0.f;

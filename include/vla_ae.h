@@ -152,6 +152,7 @@ void vla_ae_destroy(vla_ae_t h);
 #define VLA_AE_Q_OP_BYTES 6           /* algorithmic bytes one launch of loop kernel `arg` reads from HBM:
                                          the weight matrix (+ fp8 scales) of op 0 qkv, 2 o, 3 gate/up,
                                          4 down; the layer's prefix K+V for op 1 (attention) */
+#define VLA_AE_Q_ENGINE 7             /* layer engine in use: VLA_AE_ENGINE_PER_OP or VLA_AE_ENGINE_PERSISTENT */
 /* Query a property of the handle into *value.  Errors: EINVAL. */
 int vla_ae_query(vla_ae_t h, int what, int arg, long long *value);
 
@@ -162,6 +163,20 @@ int vla_ae_query(vla_ae_t h, int what, int arg, long long *value);
  * kernel with CUDA events on `stream`; weights of successive layers are distinct, so they stream
  * from HBM.  Asynchronous.  Errors: EINVAL, ENOPREFIX, ECUDA. */
 int vla_ae_bench_op(vla_ae_t h, int op, int count, int steps, void *stream);
+
+/* ------------------------------------------------------------------ layer engines
+ * How the L layers of one Euler step run (the arithmetic and its order are the same):
+ *   VLA_AE_ENGINE_PER_OP (0): five kernels per layer (QKV GEMM, attention, o-proj GEMM, gate/up
+ *     GEMM, down GEMM) chained by programmatic dependent launch;
+ *   VLA_AE_ENGINE_PERSISTENT (1): one kernel per step with one CTA per SM resident for all
+ *     layers; weights stream continuously and phases hand over through device-scope counters.
+ *     Available for bf16 weights with at most 128 token rows (batch x self tokens) when the
+ *     work units fit the SMs; create selects it whenever it is available.
+ * Select the engine for later denoise / debug calls (a graph captured for the other engine is
+ * re-captured).  Errors: EINVAL, EUNSUPPORTED (persistent engine not available here). */
+#define VLA_AE_ENGINE_PER_OP 0
+#define VLA_AE_ENGINE_PERSISTENT 1
+int vla_ae_set_engine(vla_ae_t h, int engine);
 
 /* ------------------------------------------------------------------ test hooks
  * Teacher-forced execution of one DiT layer (per-layer parity): h_in and h_out are device fp32

@@ -40,8 +40,10 @@ def _teacher_forced(c, step, layers):
 
 @pytest.mark.parametrize("name", ["starvla", "pi05"])
 def test_full_size_bf16(name):
+    import flow_matching_action_euler_b200 as fm
     c = Case(config(name))
     try:
+        assert c.ae.engine == fm.ENGINE_PERSISTENT   # what the benchmark times at batch 1
         got = c.denoise()
         ref = c.oracle_denoise()
         assert rel_err(got, ref) <= 2e-2
@@ -49,6 +51,12 @@ def test_full_size_bf16(name):
         for step in (0, c.d.steps - 1):
             errs = _teacher_forced(c, step, [0, L // 2, L - 1])
             assert max(errs.values()) <= 1e-2, (step, errs)
+        # the per-op engine on the same handle
+        c.ae.set_engine(fm.ENGINE_PER_OP)
+        per_op = c.denoise()
+        assert rel_err(per_op, ref) <= 2e-2
+        assert max(_teacher_forced(c, 0, [L - 1]).values()) <= 1e-2
+        c.ae.set_engine(fm.ENGINE_PERSISTENT)
         # velocity at step 0 (x_0 = noise)
         import torch
         x0 = oracle.bf16_to_f64(c.x["noise"])

@@ -6,6 +6,8 @@ fp8 weights <= 5e-2 on the final actions against the bf16-weight oracle and <= 2
 oracle on the dequantised weights.  Packing and fp8 codes are compared bit for bit.
 """
 
+from contextlib import contextmanager
+
 import numpy as np
 import pytest
 import torch
@@ -46,6 +48,20 @@ def case(name, **kw):
             d = d.replace(**extra)
         _cases[key] = Case(d, n_prefix=kw.get("n_prefix"), max_prefix=kw.get("max_prefix"))
     return _cases[key]
+
+
+@contextmanager
+def engine(c, which):
+    """Run the block on layer engine `which` (0 per-op kernels, 1 persistent kernel)."""
+    prev = c.ae.engine
+    c.ae.set_engine(which)
+    try:
+        yield
+    finally:
+        c.ae.set_engine(prev)
+
+
+ENGINES = [pytest.param(0, id="per_op"), pytest.param(1, id="persistent")]
 
 
 def teardown_module():
@@ -108,20 +124,24 @@ def _layer_check(c, step, steps, layers=None, tol=LAYER_TOL):
     return worst
 
 
+@pytest.mark.parametrize("eng", ENGINES)
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
-def test_layer_teacher_forced_small(name):
+def test_layer_teacher_forced_small(name, eng):
     c = case(name)
-    _layer_check(c, 0, c.d.steps)
-    _layer_check(c, c.d.steps - 1, c.d.steps)
+    with engine(c, eng):
+        _layer_check(c, 0, c.d.steps)
+        _layer_check(c, c.d.steps - 1, c.d.steps)
 
 
-def test_velocity_step0_small():
+@pytest.mark.parametrize("eng", ENGINES)
+def test_velocity_step0_small(eng):
     for name in ("tiny", "ragged"):
         c = case(name)
         d = c.d
         x0 = np.stack([c.sample_inputs(b)[0] for b in range(d.batch)])
         v = torch.empty(x0.shape, dtype=torch.float32, device="cuda")
-        c.ae.debug_velocity(0, d.steps, torch.tensor(x0, dtype=torch.float32, device="cuda"), v)
+        with engine(c, eng):
+            c.ae.debug_velocity(0, d.steps, torch.tensor(x0, dtype=torch.float32, device="cuda"), v)
         ref = []
         for b in range(d.batch):
             noise, st, kp, vp = c.sample_inputs(b)
@@ -137,6 +157,34 @@ def test_denoise_small(name):
     got = c.denoise()
     ref = c.oracle_denoise()
     assert rel_err(got, ref) <= FINAL_TOL
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_engines_agree(name):
+    """Both layer engines reach the oracle; they sum the same products in different orders."""
+    c = case(name)
+    ref = c.oracle_denoise()
+    with engine(c, 1):
+        persistent = c.denoise()
+    with engine(c, 0):
+        per_op = c.denoise()
+    assert rel_err(persistent, ref) <= FINAL_TOL
+    assert rel_err(per_op, ref) <= FINAL_TOL
+    assert rel_err(persistent, per_op) <= 1e-3
+
+
+def test_engine_selection():
+    import flow_matching_action_euler_b200 as fm
+    assert case("tiny").ae.engine == fm.ENGINE_PERSISTENT          # bf16, one n-tile: the default
+    assert case("tiny", batch=16).ae.engine == fm.ENGINE_PER_OP    # 256 token rows: per-op kernels
+    c8 = case("tiny", wtype="fp8_e4m3")
+    assert c8.ae.engine == fm.ENGINE_PER_OP
+    with pytest.raises(fm.VlaAeError) as e:
+        c8.ae.set_engine(fm.ENGINE_PERSISTENT)
+    assert e.value.code == fm.EUNSUPPORTED
+    with pytest.raises(fm.VlaAeError) as e:
+        c8.ae.set_engine(7)
+    assert e.value.code == fm.EINVAL
 
 
 def test_denoise_is_deterministic_across_replays():
