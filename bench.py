@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--euler-steps", type=int, default=None, help="Euler steps per loop (default: workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e / per-kernel timing (profiling runs)")
+    ap.add_argument("--engine", choices=("default", "per_op", "persistent"), default="default",
+                    help="layer engine: one kernel per op (the library default) or one persistent kernel per step")
     return ap.parse_args()
 
 
@@ -301,6 +303,9 @@ def run_native(args):
     vdev = torch.from_numpy(x["v"].view(np.int16)).cuda()
     sdev = torch.from_numpy(x["state"].view(np.int16)).cuda() if d.has_state_token else None
     ae.set_prefix(kdev, vdev, d.n_prefix, sdev, on_device=True, stream=stream)
+    if args.engine != "default":
+        ae.set_engine(fm.ENGINE_PERSISTENT if args.engine == "persistent" else fm.ENGINE_PER_OP)
+    engine = "persistent" if ae.engine == fm.ENGINE_PERSISTENT else "per_op"
     noise = torch.from_numpy(x["noise"].view(np.int16)).cuda()
     out = torch.empty((d.batch, d.n_action_tokens, d.action_dim), dtype=torch.float32, device="cuda")
     N = d.steps
@@ -348,7 +353,7 @@ def run_native(args):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if d.wtype == "bf16" else "e4m3 weights x bf16 activations",
-        "data": "synthetic", "config": workload_config(d, args),
+        "data": "synthetic", "config": {**workload_config(d, args), "engine": engine},
         "ms_per_loop": round(ms, 5),
         "actions_per_s": round(world * d.batch * d.n_action_tokens * 1000.0 / ms, 1),
         "chunks_per_s": round(world * d.batch * 1000.0 / ms, 2),
@@ -359,6 +364,27 @@ def run_native(args):
     }
 
     if not args.no_extras:
+        # both layer engines on the same handle and inputs (context: the line's value is `engine`'s)
+        engines = {}
+        for name, eid in (("per_op", fm.ENGINE_PER_OP), ("persistent", fm.ENGINE_PERSISTENT)):
+            try:
+                ae.set_engine(eid)
+            except fm.VlaAeError:
+                continue
+            for _ in range(3):
+                ae.denoise(noise, N, out, stream)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(10, min(args.steps, 50))
+            a.record(stream)
+            for _ in range(reps):
+                ae.denoise(noise, N, out, stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            engines[name] = {"ms_per_loop": round(a.elapsed_time(b) / reps, 4),
+                             "kernels_per_loop": int(ae.query(fm.Q_KERNELS_PER_LOOP, N))}
+        ae.set_engine(fm.ENGINE_PERSISTENT if engine == "persistent" else fm.ENGINE_PER_OP)
+        line["engines"] = engines
         # per-kernel timing through the bench hook: PDL-chained launches over successive layers
         L = d.n_layers
         count = 4 * L

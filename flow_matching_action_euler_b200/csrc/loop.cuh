@@ -485,9 +485,10 @@ __global__ void __launch_bounds__(kLoopThreads, 1) loop_kernel(const __grid_cons
             tc_fence_after();
             float* dst = p.gpart + (size_t)(u.mg * o.S + u.r) * p.gpart_unit;
             const int rows = u.nmt * 128;
+            const int ncols = min(NT, p.Ntok);   // token columns past Ntok are padding: not stored
             for (int j = 0; j < u.nmt; ++j) {
               const int row = j * 128 + quarter * 32 + lane;
-              for (int c0 = 0; c0 < NT; c0 += 16) {
+              for (int c0 = 0; c0 < ncols; c0 += 16) {
                 float vh[16], vl[16];
                 const uint32_t ta = tmem_d + (uint32_t)(buf * p.acc_cols) + ((uint32_t)(quarter * 32) << 16) +
                                     (uint32_t)(j * 2 * NT + c0);
@@ -495,7 +496,8 @@ __global__ void __launch_bounds__(kLoopThreads, 1) loop_kernel(const __grid_cons
                 tmem_ld16(ta + (uint32_t)NT, vl);
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 16; ++c) __stcg(dst + (size_t)(c0 + c) * rows + row, vh[c] + vl[c]);
+                for (int c = 0; c < 16; ++c)
+                  if (c0 + c < ncols) __stcg(dst + (size_t)(c0 + c) * rows + row, vh[c] + vl[c]);
               }
             }
             tc_fence_before();

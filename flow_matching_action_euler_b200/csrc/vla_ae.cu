@@ -434,7 +434,7 @@ LoopKernel loop_kernel_for(int hd, int cs) {
 int plan_loop(vla_ae* H) {
   const vla_ae_dims& d = H->d;
   H->loop_ok = false;
-  if (H->fp8 || H->Nt != 1 || H->NT > 128) return VLA_AE_OK;
+  if (H->fp8 || H->Nt != 1 || H->NT > 128 || d.hidden % 4 != 0) return VLA_AE_OK;
   const int G = H->num_sms, NT = H->NT, hd = d.head_dim;
   LoopParams lp{};
   const OpId ids[4] = {OP_QKV, OP_O, OP_GU, OP_D};
@@ -443,8 +443,9 @@ int plan_loop(vla_ae* H) {
   const int nrb = ceil_div(rep * H->Ts, kAttnRows);
   const int groups = nrb * d.n_kv_heads * d.batch;
   const int Lmax = d.max_prefix + H->Ts;
-  // key spans: up to 8 per block (one round of loads per merged value), as many as the SMs allow
-  const int S0 = std::max(1, std::min({Lmax, 8, G / groups}));
+  // key spans: up to 16 per block (at most two rounds of loads per merged value), as many as
+  // the SMs allow; a span's own time grows with its length
+  const int S0 = std::max(1, std::min({Lmax, 16, G / groups}));
   const int span = (int)align_up((size_t)ceil_div(Lmax, S0), 16);
   const int attn_S = ceil_div(Lmax, span);
   const int cs = span <= 16 ? 16 : 32;
@@ -588,8 +589,7 @@ int plan_loop(vla_ae* H) {
   if ((rc = H->alloc(&H->loop_dbg_ctr, H->ctr_step * 4))) return rc;
   H->loop_cs = cs;
   H->loop_proto = lp;
-  H->loop_ok = true;
-  H->use_loop = true;
+  H->loop_ok = true;   // available; the per-op engine stays the default (it measures faster)
   return VLA_AE_OK;
 }
 

@@ -170,8 +170,9 @@ int vla_ae_bench_op(vla_ae_t h, int op, int count, int steps, void *stream);
  *     GEMM, down GEMM) chained by programmatic dependent launch;
  *   VLA_AE_ENGINE_PERSISTENT (1): one kernel per step with one CTA per SM resident for all
  *     layers; weights stream continuously and phases hand over through device-scope counters.
- *     Available for bf16 weights with at most 128 token rows (batch x self tokens) when the
- *     work units fit the SMs; create selects it whenever it is available.
+ *     Available for bf16 weights with at most 128 token rows (batch x self tokens), a hidden
+ *     size that is a multiple of 4, and work units that fit the SMs.
+ * create selects VLA_AE_ENGINE_PER_OP.
  * Select the engine for later denoise / debug calls (a graph captured for the other engine is
  * re-captured).  Errors: EINVAL, EUNSUPPORTED (persistent engine not available here). */
 #define VLA_AE_ENGINE_PER_OP 0

@@ -43,7 +43,8 @@ def test_full_size_bf16(name):
     import flow_matching_action_euler_b200 as fm
     c = Case(config(name))
     try:
-        assert c.ae.engine == fm.ENGINE_PERSISTENT   # what the benchmark times at batch 1
+        assert c.ae.engine == fm.ENGINE_PER_OP       # the default, what the benchmark times
+        c.ae.set_engine(fm.ENGINE_PERSISTENT)
         got = c.denoise()
         ref = c.oracle_denoise()
         assert rel_err(got, ref) <= 2e-2
@@ -55,8 +56,8 @@ def test_full_size_bf16(name):
         c.ae.set_engine(fm.ENGINE_PER_OP)
         per_op = c.denoise()
         assert rel_err(per_op, ref) <= 2e-2
+        assert rel_err(per_op, got) <= 5e-3
         assert max(_teacher_forced(c, 0, [L - 1]).values()) <= 1e-2
-        c.ae.set_engine(fm.ENGINE_PERSISTENT)
         # velocity at step 0 (x_0 = noise)
         import torch
         x0 = oracle.bf16_to_f64(c.x["noise"])

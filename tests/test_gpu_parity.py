@@ -175,8 +175,14 @@ def test_engines_agree(name):
 
 def test_engine_selection():
     import flow_matching_action_euler_b200 as fm
-    assert case("tiny").ae.engine == fm.ENGINE_PERSISTENT          # bf16, one n-tile: the default
-    assert case("tiny", batch=16).ae.engine == fm.ENGINE_PER_OP    # 256 token rows: per-op kernels
+    c = case("tiny")
+    assert c.ae.engine == fm.ENGINE_PER_OP                        # the default
+    with engine(c, fm.ENGINE_PERSISTENT):                          # bf16, one n-tile: available
+        assert c.ae.engine == fm.ENGINE_PERSISTENT
+    c16 = case("tiny", batch=16)                                   # 256 token rows: per-op only
+    with pytest.raises(fm.VlaAeError) as e:
+        c16.ae.set_engine(fm.ENGINE_PERSISTENT)
+    assert e.value.code == fm.EUNSUPPORTED
     c8 = case("tiny", wtype="fp8_e4m3")
     assert c8.ae.engine == fm.ENGINE_PER_OP
     with pytest.raises(fm.VlaAeError) as e:
