@@ -14,6 +14,10 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
 =====================  =========================================================
 ``euler_integrate``    closed form of Euler on a linear field v = A x + b,
                        exact-ODE error bound, A = 0 and N = 1 special cases
+``euler_integrate_grid`` the uniform grid reproduces ``euler_integrate``; a
+                       skipped-step grid equals a brute-force velocity cache
+                       (DP-Cache reading); first-order convergence on a graded
+                       grid; the one-step grid; grid validation
 ``timestep_embedding`` t = 0 gives [1..1, 0..0]; first frequency is 1000 t;
                        last frequency matches the base-10000 geometric series
 ``rms_norm``           unit RMS at eps = 0, scale invariance, torch's rms_norm
@@ -33,7 +37,8 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
 
 from .model import (  # noqa: F401
     bf16_to_f64, t_schedule, timestep_embedding, silu, rms_norm, modulate, rope_half,
-    rope_positions_angles, gqa_attention, linear, swiglu, euler_integrate,
+    rope_positions_angles, gqa_attention, linear, swiglu, euler_integrate, euler_integrate_grid,
+    check_t_grid, uniform_grid,
     adaln_table, dit_layer, embed_tokens, velocity, denoise, denoise_batch, OracleWeights,
 )
 from .fp8 import (  # noqa: F401

@@ -44,6 +44,39 @@ def t_schedule(n_steps: int):
     return [1.0 - k / n_steps for k in range(n_steps)], -1.0 / n_steps
 
 
+def check_t_grid(t_grid) -> List[float]:
+    """A time grid t_0 > t_1 > ... > t_n (n >= 1, finite values) as floats.
+
+    Step skipping ("跨XPU平台表征视觉-语言-动作模型" sections 5.2 and 5.3.2: DP-Cache drops a fixed set
+    of intermediate diffusion steps) and the one-step variant (APXInf article, section "CUDA
+    Graph、FP8 和 Rust") are such grids: a dropped step's interval joins the step before it, which
+    for Euler is the same as reusing that step's velocity over the dropped interval."""
+    g = [float(t) for t in t_grid]
+    if len(g) < 2:
+        raise ValueError("a time grid needs at least two points")
+    if not all(math.isfinite(t) for t in g):
+        raise ValueError("time grid values must be finite")
+    if not all(b < a for a, b in zip(g, g[1:])):
+        raise ValueError("time grid must be strictly decreasing")
+    return g
+
+
+def uniform_grid(n_steps: int) -> List[float]:
+    """t_k = 1 - k/N for k = 0..N (t_N = 0): the grid of the fixed-step loop."""
+    if n_steps < 1:
+        raise ValueError("n_steps must be >= 1")
+    return [1.0 - k / n_steps for k in range(n_steps + 1)]
+
+
+def euler_integrate_grid(x0: np.ndarray, t_grid, v_fn: Callable[[np.ndarray, float], np.ndarray]) -> np.ndarray:
+    """Explicit Euler along a time grid: x_{k+1} = x_k + (t_{k+1} - t_k) * v(x_k, t_k)."""
+    g = check_t_grid(t_grid)
+    x = np.array(x0, dtype=np.float64, copy=True)
+    for t0, t1 in zip(g, g[1:]):
+        x = x + (t1 - t0) * v_fn(x, t0)
+    return x
+
+
 def euler_integrate(x0: np.ndarray, n_steps: int, v_fn: Callable[[np.ndarray, float], np.ndarray]) -> np.ndarray:
     """Fixed-step explicit Euler from t = 1 to t = 0: x_{k+1} = x_k + dt * v(x_k, t_k)."""
     ts, dt = t_schedule(n_steps)
@@ -234,15 +267,18 @@ def velocity(x: np.ndarray, t: float, state: Optional[np.ndarray], W: OracleWeig
 
 
 def denoise(noise: np.ndarray, state: Optional[np.ndarray], W: OracleWeights, k_prefix: np.ndarray,
-            v_prefix: np.ndarray, d, n_steps: int) -> np.ndarray:
-    """x_N of the N-step Euler loop for one sample (inputs already float64)."""
-    return euler_integrate(noise, n_steps,
-                           lambda x, t: velocity(x, t, state, W, k_prefix, v_prefix, d))
+            v_prefix: np.ndarray, d, n_steps: int, t_grid=None) -> np.ndarray:
+    """x_N of the N-step Euler loop for one sample (inputs already float64); with `t_grid`, the
+    Euler loop along that time grid instead (n_steps is then ignored)."""
+    v_fn = lambda x, t: velocity(x, t, state, W, k_prefix, v_prefix, d)
+    if t_grid is not None:
+        return euler_integrate_grid(noise, t_grid, v_fn)
+    return euler_integrate(noise, n_steps, v_fn)
 
 
 def denoise_batch(weights_bits: Dict[str, object], inputs_bits: Dict[str, np.ndarray], d,
                   n_steps: Optional[int] = None, samples: Optional[List[int]] = None,
-                  W: Optional[OracleWeights] = None) -> np.ndarray:
+                  W: Optional[OracleWeights] = None, t_grid=None) -> np.ndarray:
     """Run ``denoise`` per sample on the synthetic bf16 inputs; returns [len(samples), T, A]."""
     n_steps = d.steps if n_steps is None else n_steps
     if W is None:
@@ -255,5 +291,5 @@ def denoise_batch(weights_bits: Dict[str, object], inputs_bits: Dict[str, np.nda
         state = bf16_to_f64(inputs_bits["state"][b]) if d.has_state_token else None
         kp = bf16_to_f64(inputs_bits["k"][b])
         vp = bf16_to_f64(inputs_bits["v"][b])
-        outs.append(denoise(noise, state, W, kp, vp, d, n_steps))
+        outs.append(denoise(noise, state, W, kp, vp, d, n_steps, t_grid=t_grid))
     return np.stack(outs)

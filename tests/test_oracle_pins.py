@@ -88,6 +88,68 @@ def test_euler_time_grid_golden():
         np.testing.assert_allclose(seen, ts, rtol=0, atol=1e-15)
 
 
+# ----------------------------------------------------------------- Euler along a time grid
+
+def test_euler_grid_uniform_matches_fixed_step():
+    a, b, x0 = _linear_field(seed=7)
+    for n in (1, 3, 10):
+        got = oracle.euler_integrate_grid(x0, oracle.uniform_grid(n), lambda x, t: a @ x + b + t)
+        want = oracle.euler_integrate(x0, n, lambda x, t: a @ x + b + t)
+        np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+
+
+def test_euler_grid_skipping_equals_velocity_cache():
+    """Dropping grid points = reusing the last computed velocity over the dropped steps."""
+    a, b, x0 = _linear_field(seed=8)
+    field = lambda x, t: np.tanh(a @ x) + b * t
+    n = 10
+    keep = {0, 1, 2, 6, 9}                      # velocities recomputed only at these steps
+    x, v = np.array(x0), None
+    for k in range(n):                           # brute force: the uniform loop with a cache
+        if k in keep:
+            v = field(x, 1.0 - k / n)
+        x = x + (-1.0 / n) * v
+    grid = [1.0 - k / n for k in sorted(keep)] + [0.0]
+    got = oracle.euler_integrate_grid(x0, grid, field)
+    np.testing.assert_allclose(got, x, rtol=1e-13, atol=1e-13)
+
+
+def test_euler_grid_converges_first_order_on_a_graded_grid():
+    a, b, x0 = _linear_field(seed=3)
+    ea = scipy.linalg.expm(-a)
+    exact = ea @ x0 + np.linalg.solve(a, (ea - np.eye(7)) @ b)
+    errs = []
+    for n in (64, 128, 256):
+        grid = [(1.0 - k / n) ** 2 for k in range(n + 1)]      # steps from 2/n down to 1/n^2
+        errs.append(np.max(np.abs(oracle.euler_integrate_grid(x0, grid, lambda x, t: a @ x + b) - exact)))
+    for r in (errs[0] / errs[1], errs[1] / errs[2]):
+        assert 1.8 < r < 2.2, errs
+
+
+def test_euler_grid_one_step_and_order_of_times():
+    _, b, x0 = _linear_field(seed=9)
+    seen = []
+
+    def v(x, t):
+        seen.append(t)
+        return np.cos(x) * t
+
+    got = oracle.euler_integrate_grid(x0, [1.0, 0.0], v)
+    assert seen == [1.0]
+    assert np.array_equal(got, x0 - np.cos(x0))
+    seen.clear()
+    oracle.euler_integrate_grid(x0, [0.9, 0.7, 0.2, -0.1], v)
+    assert seen == [0.9, 0.7, 0.2]
+    got = oracle.euler_integrate_grid(x0, [1.0, 0.6, 0.25, 0.0], lambda x, t: b)
+    np.testing.assert_allclose(got, x0 - b, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("grid", [[1.0], [1.0, 1.0], [0.2, 0.5], [1.0, float("nan"), 0.0], [1.0, 0.5, 0.5, 0.0]])
+def test_euler_grid_rejects_bad_grids(grid):
+    with pytest.raises(ValueError):
+        oracle.check_t_grid(grid)
+
+
 # ----------------------------------------------------------------- time embedding
 
 def test_timestep_embedding_t0_and_identity():
