@@ -126,9 +126,9 @@ __global__ void __launch_bounds__(kTailThreads) tail_kernel(const __grid_constan
 
 // ---------------------------------------------------------------- input-independent tables
 // c_k = SiLU(temb(t_k)), temb(t) = [cos(a_i), sin(a_i)], a_i = 1000 t 10000^(-i/half), in double.
-__global__ void temb_kernel(double* c, int steps, int dt_dim) {
+__global__ void temb_kernel(const double* __restrict__ ts, double* c, int dt_dim) {
   const int k = blockIdx.x, half = dt_dim / 2;
-  const double t = 1.0 - (double)k / (double)steps;
+  const double t = ts[k];
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
     const double a = 1000.0 * t * exp(-log(10000.0) * (double)i / (double)half);
     const double cs = cos(a), sn = sin(a);

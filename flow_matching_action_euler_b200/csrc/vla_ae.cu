@@ -64,6 +64,8 @@ struct StepTables {
   float* cq = nullptr;     // [steps][L][Mt_qkv * 128]: W_qkv . shift_attn
   float* cg = nullptr;     // [steps][L][Mt_gu * 128]:  W_gu . shift_mlp
   unsigned* ctr = nullptr;  // persistent engine: per-step counter blocks [steps][ctr_step]
+  std::vector<double> t;    // time grid t_0 > ... > t_steps
+  std::vector<float> dt;    // Euler step k: t_{k+1} - t_k
   cudaGraphExec_t exec = nullptr;
   int captured_prefix = -1;
   int captured_engine = -1;
@@ -102,7 +104,7 @@ struct vla_ae {
   size_t device_bytes = 0;
   int n_prefix = -1;
   cudaStream_t cap = nullptr;
-  std::map<int, StepTables> tables;
+  std::map<std::vector<double>, StepTables> tables;   // keyed by the time grid
 
   template <typename T>
   int alloc(T** p, size_t bytes) {
@@ -857,7 +859,7 @@ cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
       t.ss_parts = ss_parts_final(H);
       t.shift_f = T.fmod + (size_t)k * 2 * H->d.hidden;
       t.scale_f = t.shift_f + H->d.hidden;
-      t.dt = -1.0f / (float)N;
+      t.dt = T.dt[k];
       t.do_out = 1;
       t.do_in = k + 1 < N;
       if (t.do_in) t.sc_next = layer_mod(H, T, k + 1, 0).scale_a;
@@ -881,7 +883,7 @@ cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
     t.ss_parts = ss_parts_of(H, OP_D);
     t.shift_f = T.fmod + (size_t)k * 2 * H->d.hidden;
     t.scale_f = t.shift_f + H->d.hidden;
-    t.dt = -1.0f / (float)N;
+    t.dt = T.dt[k];
     t.do_out = 1;
     t.do_in = k + 1 < N;
     if (t.do_in) t.sc_next = layer_mod(H, T, k + 1, 0).scale_a;
@@ -891,22 +893,32 @@ cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
   return cudaSuccess;
 }
 
-int get_tables(vla_ae* H, int steps, StepTables** out) {
-  auto it = H->tables.find(steps);
+// The tables of one time grid (t_0 > ... > t_n): adaLN modulation per (step, layer), the final
+// modulation, the W . shift tables, the per-step dt and the persistent engine's counters.
+// `uniform`: the grid of vla_ae_denoise (t_k = 1 - k/N), whose step is exactly -1/N.
+int get_tables_grid(vla_ae* H, const std::vector<double>& grid, bool uniform, StepTables** out) {
+  auto it = H->tables.find(grid);
   if (it != H->tables.end()) {
     *out = &it->second;
     return VLA_AE_OK;
   }
+  const int steps = (int)grid.size() - 1;
   StepTables T;
   T.steps = steps;
+  T.t = grid;
+  T.dt.resize(steps);
+  for (int k = 0; k < steps; ++k) T.dt[k] = uniform ? -1.0f / (float)steps : (float)(grid[k + 1] - grid[k]);
   const vla_ae_dims& d = H->d;
   const size_t Hd = d.hidden;
   int rc;
   if ((rc = H->alloc(&T.mod, (size_t)steps * d.n_layers * 6 * Hd * 4))) return rc;
   if ((rc = H->alloc(&T.fmod, (size_t)steps * 2 * Hd * 4))) return rc;
   double* c = nullptr;
+  double* tdev = nullptr;
   CK(cudaMalloc(&c, (size_t)steps * d.t_emb_dim * sizeof(double)));
-  temb_kernel<<<steps, 128, 0, H->cap>>>(c, steps, d.t_emb_dim);
+  CK(cudaMalloc(&tdev, (size_t)steps * sizeof(double)));
+  CK(cudaMemcpy(tdev, grid.data(), (size_t)steps * sizeof(double), cudaMemcpyHostToDevice));
+  temb_kernel<<<steps, 128, 0, H->cap>>>(tdev, c, d.t_emb_dim);
   for (int l = 0; l < d.n_layers; ++l) {
     const int rows = 6 * d.hidden;
     adaln_table_kernel<<<ceil_div(rows, 8), 256, 0, H->cap>>>(H->w_ada + (size_t)l * rows * d.t_emb_dim,
@@ -939,10 +951,19 @@ int get_tables(vla_ae* H, int steps, StepTables** out) {
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(H->cap));
   CK(cudaFree(c));
-  auto res = H->tables.emplace(steps, T);
+  CK(cudaFree(tdev));
+  auto res = H->tables.emplace(grid, T);
   *out = &res.first->second;
   return VLA_AE_OK;
 }
+
+std::vector<double> uniform_grid(int steps) {
+  std::vector<double> g(steps + 1);
+  for (int k = 0; k <= steps; ++k) g[k] = 1.0 - (double)k / (double)steps;
+  return g;
+}
+
+int get_tables(vla_ae* H, int steps, StepTables** out) { return get_tables_grid(H, uniform_grid(steps), true, out); }
 
 int ensure_graph(vla_ae* H, StepTables* T) {
   if (T->exec && T->captured_prefix == H->n_prefix && T->captured_engine == (int)H->use_loop) return VLA_AE_OK;
@@ -1197,13 +1218,9 @@ int vla_ae_set_prefix(vla_ae_t H, const void* k, const void* v, int n_prefix, co
   return VLA_AE_OK;
 }
 
-static int denoise_common(vla_ae_t H, const void* noise, int steps, float* out, void* stream, bool host) {
-  if (!H || !noise || !out || steps < 1) return VLA_AE_EINVAL;
-  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+static int denoise_tables(vla_ae_t H, StepTables* T, const void* noise, float* out, void* stream, bool host) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  StepTables* T = nullptr;
-  int rc = get_tables(H, steps, &T);
-  if (rc) return rc;
+  int rc;
   if ((rc = ensure_graph(H, T))) return rc;
   const vla_ae_dims& d = H->d;
   const size_t nx = (size_t)d.batch * d.n_action_tokens * d.action_dim;
@@ -1213,12 +1230,35 @@ static int denoise_common(vla_ae_t H, const void* noise, int steps, float* out, 
   return VLA_AE_OK;
 }
 
+static int denoise_common(vla_ae_t H, const void* noise, int steps, float* out, void* stream, bool host) {
+  if (!H || !noise || !out || steps < 1) return VLA_AE_EINVAL;
+  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+  StepTables* T = nullptr;
+  int rc = get_tables(H, steps, &T);
+  if (rc) return rc;
+  return denoise_tables(H, T, noise, out, stream, host);
+}
+
 int vla_ae_denoise(vla_ae_t H, const void* noise, int steps, float* out, void* stream) {
   return denoise_common(H, noise, steps, out, stream, false);
 }
 
 int vla_ae_denoise_host(vla_ae_t H, const void* noise_host, int steps, float* out_host, void* stream) {
   return denoise_common(H, noise_host, steps, out_host, stream, true);
+}
+
+int vla_ae_denoise_sched(vla_ae_t H, const void* noise, const float* t_grid, int n, float* out, void* stream) {
+  if (!H || !noise || !out || !t_grid || n < 1 || n > VLA_AE_MAX_GRID_STEPS) return VLA_AE_EINVAL;
+  std::vector<double> grid(n + 1);
+  for (int k = 0; k <= n; ++k) {
+    grid[k] = (double)t_grid[k];
+    if (!std::isfinite(grid[k]) || (k > 0 && !(grid[k] < grid[k - 1]))) return VLA_AE_EINVAL;
+  }
+  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+  StepTables* T = nullptr;
+  int rc = get_tables_grid(H, grid, false, &T);
+  if (rc) return rc;
+  return denoise_tables(H, T, noise, out, stream, false);
 }
 
 int vla_ae_status(vla_ae_t H) {

@@ -128,6 +128,19 @@ int vla_ae_set_prefix_static(vla_ae_t h, const void *k, const void *v, int n_pre
  * `stream`.  Errors: EINVAL, ENOPREFIX, ECUDA. */
 int vla_ae_denoise(vla_ae_t h, const void *noise, int steps, float *out, void *stream);
 
+/* The Euler loop along a caller-chosen time grid: n steps x_{k+1} = x_k + (t_{k+1} - t_k) *
+ * v(x_k, t_k) for the host array t_grid[0..n] (strictly decreasing, finite; 1 <= n <=
+ * VLA_AE_MAX_GRID_STEPS).  It serves step skipping ("跨XPU平台表征视觉-语言-动作模型" sections 5.2
+ * and 5.3.2: DP-Cache drops a fixed set of intermediate diffusion steps; for Euler a dropped
+ * step's interval joining the step before it equals reusing that step's velocity) and the
+ * one-step variant (APXInf article, section "CUDA Graph、FP8 和 Rust"): {1, 0}.
+ *   noise  device bf16 [B][T][A];  out  device fp32 [B][T][A] (caller-owned).
+ * The first call for a given grid builds its tables and captures its graph (as vla_ae_denoise
+ * does per step count; the uniform grid with values exactly 1 - k/n shares that step count's
+ * tables).  Asynchronous on `stream`.  Errors: EINVAL (bad grid or pointers), ENOPREFIX, ECUDA. */
+#define VLA_AE_MAX_GRID_STEPS 256
+int vla_ae_denoise_sched(vla_ae_t h, const void *noise, const float *t_grid, int n, float *out, void *stream);
+
 /* Same as vla_ae_denoise with host buffers: noise_host bf16 [B][T][A] and out_host fp32
  * [B][T][A] (pinned memory gives asynchronous copies).  Enqueues the host-to-device copy, the
  * loop and the device-to-host copy on `stream`; out_host is valid after the stream syncs. */

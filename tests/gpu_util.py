@@ -47,9 +47,9 @@ class Case:
         assert self.ae.status() == 0
         return out.cpu().numpy()
 
-    def oracle_denoise(self, steps: int | None = None, samples=None, W=None) -> np.ndarray:
+    def oracle_denoise(self, steps: int | None = None, samples=None, W=None, t_grid=None) -> np.ndarray:
         return oracle.denoise_batch(self.w, self.x, self.d, n_steps=steps, samples=samples,
-                                    W=self.W if W is None else W)
+                                    W=self.W if W is None else W, t_grid=t_grid)
 
     def sample_inputs(self, b: int):
         x = self.x

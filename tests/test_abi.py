@@ -98,6 +98,9 @@ def test_null_arguments(fm):
     assert fm.vla_ae_debug_weight(None, 0, 0, None, None) == fm.EINVAL
     assert fm.vla_ae_debug_wait_probe(None, 10) == fm.EINVAL
     assert fm.vla_ae_set_prefix_static(None, None, None, 0, None, None) == fm.EINVAL
+    g = (ctypes.c_float * 3)(1.0, 0.5, 0.0)
+    assert fm.vla_ae_denoise_sched(None, None, g, 2, None, None) == fm.EINVAL
+    assert fm.vla_ae_set_engine(None, fm.ENGINE_PER_OP) == fm.EINVAL
     fm.vla_ae_destroy(None)   # no-op
 
 

@@ -83,6 +83,23 @@ def test_full_size_fp8(steps):
         c.close()
 
 
+def test_pi05_one_step_variant():
+    """The one-step action generation of the APXInf article on the pi0.5 shape: grid {1, 0}."""
+    import torch
+    c = Case(config("pi05"))
+    try:
+        noise = torch.from_numpy(c.x["noise"].view(np.int16)).cuda()
+        out = torch.empty((1, c.d.n_action_tokens, c.d.action_dim), dtype=torch.float32, device="cuda")
+        c.ae.denoise_sched(noise, [1.0, 0.0], out)
+        torch.cuda.synchronize()
+        assert c.ae.status() == 0
+        ref = c.oracle_denoise(t_grid=[1.0, 0.0])
+        assert rel_err(out.cpu().numpy(), ref) <= 2e-2
+        assert np.array_equal(out.cpu().numpy(), c.denoise(1))   # the same grid as 1 uniform step
+    finally:
+        c.close()
+
+
 @pytest.mark.parametrize("batch", [4, 16, 64])
 def test_starvla_batch_sweep_sampled(batch):
     c = Case(config("starvla", batch=batch))

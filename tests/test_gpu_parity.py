@@ -193,6 +193,48 @@ def test_engine_selection():
     assert e.value.code == fm.EINVAL
 
 
+def _denoise_sched(c, grid):
+    d = c.d
+    from tests.gpu_util import bits_to_cuda
+    noise = bits_to_cuda(c.x["noise"])
+    out = torch.empty((d.batch, d.n_action_tokens, d.action_dim), dtype=torch.float32, device="cuda")
+    c.ae.denoise_sched(noise, grid, out)
+    torch.cuda.synchronize()
+    assert c.ae.status() == 0
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("eng", ENGINES)
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_denoise_time_grid(name, eng):
+    """A nonuniform grid and the one-step grid, against the oracle along the same grid."""
+    c = case(name)
+    with engine(c, eng):
+        for grid in ([1.0, 0.8, 0.35, 0.1, 0.0], [1.0, 0.0]):
+            got = _denoise_sched(c, grid)
+            ref = c.oracle_denoise(t_grid=[float(np.float32(t)) for t in grid])
+            assert rel_err(got, ref) <= FINAL_TOL, grid
+
+
+def test_denoise_time_grid_uniform_and_skipping():
+    c = case("tiny")
+    # the uniform 4-step grid is exact in fp32: the same tables and graph as vla_ae_denoise(4)
+    assert np.array_equal(_denoise_sched(c, [1.0, 0.75, 0.5, 0.25, 0.0]), c.denoise(4))
+    # DP-Cache style: velocities of a 10-step loop recomputed at steps 0, 1, 2, 6, 9 only
+    grid = [1.0, 0.9, 0.8, 0.4, 0.1, 0.0]
+    got = _denoise_sched(c, grid)
+    assert rel_err(got, c.oracle_denoise(t_grid=[float(np.float32(t)) for t in grid])) <= FINAL_TOL
+
+
+def test_denoise_time_grid_rejects_bad_grids():
+    import flow_matching_action_euler_b200 as fm
+    c = case("tiny")
+    for grid in ([1.0], [1.0, 1.0], [0.0, 1.0], [1.0, float("nan"), 0.0]):
+        with pytest.raises(fm.VlaAeError) as e:
+            _denoise_sched(c, grid)
+        assert e.value.code == fm.EINVAL
+
+
 def test_denoise_is_deterministic_across_replays():
     c = case("tiny")
     a = c.denoise()
