@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200, help="timed denoise loops")
     ap.add_argument("--warmup", type=int, default=20, help="untimed denoise loops (>= 3)")
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
-    ap.add_argument("--workload", default="starvla", choices=("starvla", "pi05", "pi05_fp8", "tiny"))
+    ap.add_argument("--workload", default="starvla", choices=("starvla", "pi05", "pi05_fp8", "pi05_int8", "tiny"))
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--euler-steps", type=int, default=None, help="Euler steps per loop (default: workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -207,7 +207,7 @@ def oracle_sample_rate(d, w, x, budget_s=10.0, per_layer=False, n_samples=None, 
     """Time the oracle on a bounded sample of the workload; returns (GB/s, seconds, description, ms/sample)."""
     import numpy as np
     import oracle
-    W = oracle.OracleWeights(w, d, quantized=(d.wtype != "bf16"))
+    W = oracle.OracleWeights(w, d, quantized=d.wtype)
     for l in range(d.n_layers):
         W.layer(l)
     noise = oracle.bf16_to_f64(x["noise"][0])
@@ -352,7 +352,8 @@ def run_native(args):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if d.wtype == "bf16" else "e4m3 weights x bf16 activations",
+        "vs_baseline": None, "dtype": {"bf16": "bf16", "fp8_e4m3": "e4m3 weights x bf16 activations",
+                  "int8": "int8 weights x bf16 activations"}[d.wtype],
         "data": "synthetic", "config": {**workload_config(d, args), "engine": engine},
         "ms_per_loop": round(ms, 5),
         "actions_per_s": round(world * d.batch * d.n_action_tokens * 1000.0 / ms, 1),

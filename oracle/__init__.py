@@ -28,6 +28,9 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
                        matrix, P = 0, constant-V rows, MHA case
 ``linear``/``swiglu``  torch float64 linear / silu, SiLU(0) = 0
 ``e4m3_*``             exhaustive code table, RNE ties, saturation, torch cast
+``*_int8``             the max entry maps to +-127, integer multiples of the
+                       scale round-trip, half-to-even ties, zero rows, torch's
+                       round on the same quotients, |W' - W| <= scale / 2
 ``dit_layer``          zero gates give the identity, joint prefix permutation
                        invariance
 ``velocity``/``denoise``  parity unpinned beyond the parts above: batch
@@ -44,3 +47,4 @@ from .model import (  # noqa: F401
 from .fp8 import (  # noqa: F401
     e4m3_decode, e4m3_encode, quantize_rowwise_e4m3, dequantize_rowwise_e4m3,
 )
+from .int8 import quantize_rowwise_int8, dequantize_rowwise_int8  # noqa: F401

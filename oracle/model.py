@@ -27,6 +27,7 @@ from typing import Callable, Dict, List, Optional
 import numpy as np
 
 from .fp8 import quantize_rowwise_e4m3, dequantize_rowwise_e4m3
+from .int8 import quantize_rowwise_int8, dequantize_rowwise_int8
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
@@ -170,16 +171,20 @@ _LAYER_LINEARS = ("wq", "wk", "wv", "wo", "wg", "wu", "wd")
 
 
 class OracleWeights:
-    """float64 view of the synthetic bf16 weights (optionally with e4m3-dequantised linears).
+    """float64 view of the synthetic bf16 weights (optionally with dequantised 8-bit linears).
 
-    ``quantized=True`` replaces each per-layer q/k/v/o/gate/up/down weight W by
-    W' = e4m3(W / s) * s with one scale per output channel; adaLN, in/out/state
-    projections stay bf16.
+    ``quantized`` = ``"fp8_e4m3"`` (or ``True``) replaces each per-layer q/k/v/o/gate/up/down
+    weight W by W' = e4m3(W / s) * s, ``"int8"`` by W' = round(W / s) * s, with one scale per
+    output channel; adaLN, in/out/state projections stay bf16.  ``False`` / ``"bf16"``: none.
     """
 
-    def __init__(self, w: Dict[str, object], d, quantized: bool = False):
+    def __init__(self, w: Dict[str, object], d, quantized=False):
         self.d = d
-        self.quantized = quantized
+        if quantized is True:
+            quantized = "fp8_e4m3"
+        self.quantized = False if quantized in (False, None, "bf16") else quantized
+        if self.quantized not in (False, "fp8_e4m3", "int8"):
+            raise ValueError(f"unknown weight format {quantized!r}")
         self._raw = w
         self.top = {k: bf16_to_f64(v) for k, v in w.items() if k != "layers"}
         self._cache: Dict[int, Dict[str, np.ndarray]] = {}
@@ -189,10 +194,14 @@ class OracleWeights:
             return self._cache[l]
         raw = self._raw["layers"][l]
         lw = {k: bf16_to_f64(v) for k, v in raw.items()}
-        if self.quantized:
+        if self.quantized == "fp8_e4m3":
             for k in _LAYER_LINEARS:
                 codes, scales = quantize_rowwise_e4m3(lw[k].astype(np.float32))
                 lw[k] = dequantize_rowwise_e4m3(codes, scales)
+        elif self.quantized == "int8":
+            for k in _LAYER_LINEARS:
+                codes, scales = quantize_rowwise_int8(lw[k].astype(np.float32))
+                lw[k] = dequantize_rowwise_int8(codes, scales)
         self._cache[l] = lw
         return lw
 
@@ -282,7 +291,7 @@ def denoise_batch(weights_bits: Dict[str, object], inputs_bits: Dict[str, np.nda
     """Run ``denoise`` per sample on the synthetic bf16 inputs; returns [len(samples), T, A]."""
     n_steps = d.steps if n_steps is None else n_steps
     if W is None:
-        W = OracleWeights(weights_bits, d, quantized=(d.wtype != "bf16"))
+        W = OracleWeights(weights_bits, d, quantized=d.wtype)
     B = inputs_bits["noise"].shape[0]
     samples = list(range(B)) if samples is None else samples
     outs = []

@@ -17,6 +17,8 @@ Workload shapes follow the five workloads the action expert is measured on:
                   32, 800 prefix tokens.
 * ``pi05_fp8`` -- ``pi05`` with e4m3 linear weights (per-output-channel
                   fp32 scales), 1 or 10 steps.
+* ``pi05_int8`` -- ``pi05`` with int8 linear weights (per-output-channel
+                  fp32 scales; the INT8 fallback of the same article).
 * batch sweep  -- ``tiny`` and ``starvla`` at batch 1, 4, 16 and 64.
 
 Random numbers: numpy's PCG64 bit generator (O'Neill, "PCG: A Family of
@@ -59,7 +61,7 @@ class Dims:
     n_prefix: int
     steps: int
     batch: int = 1
-    wtype: str = "bf16"          # "bf16" or "fp8_e4m3"
+    wtype: str = "bf16"          # "bf16", "fp8_e4m3" or "int8"
     rope_theta: float = 10000.0
     rms_eps: float = 1e-6
 
@@ -93,6 +95,9 @@ CONFIGS: Dict[str, Dims] = {
     "pi05_fp8": Dims(n_layers=18, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=256,
                      inter=4096, t_emb_dim=256, action_dim=32, n_action_tokens=50,
                      has_state_token=0, n_prefix=800, steps=10, wtype="fp8_e4m3"),
+    "pi05_int8": Dims(n_layers=18, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=256,
+                      inter=4096, t_emb_dim=256, action_dim=32, n_action_tokens=50,
+                      has_state_token=0, n_prefix=800, steps=10, wtype="int8"),
 }
 
 BATCH_SWEEP = (1, 4, 16, 64)
@@ -220,4 +225,4 @@ def abi_dims(d: Dims, max_prefix: int | None = None) -> Dict[str, object]:
                 head_dim=d.head_dim, inter=d.inter, t_emb_dim=d.t_emb_dim, action_dim=d.action_dim,
                 n_action_tokens=d.n_action_tokens, has_state_token=d.has_state_token,
                 max_prefix=d.n_prefix if max_prefix is None else max_prefix, batch=d.batch,
-                rope_theta=d.rope_theta, rms_eps=d.rms_eps, wtype=0 if d.wtype == "bf16" else 1)
+                rope_theta=d.rope_theta, rms_eps=d.rms_eps, wtype={"bf16": 0, "fp8_e4m3": 1, "int8": 2}[d.wtype])

@@ -35,7 +35,7 @@ class Case:
                                   self.w)
         self.ae.set_prefix(self.x["k"] if self.P else None, self.x["v"] if self.P else None, self.P,
                            self.x.get("state"))
-        self.W = oracle.OracleWeights(self.w, d, quantized=(d.wtype != "bf16"))
+        self.W = oracle.OracleWeights(self.w, d, quantized=d.wtype)
 
     def denoise(self, steps: int | None = None) -> np.ndarray:
         d = self.d

@@ -487,3 +487,38 @@ def test_layer_branch_isolation_under_zero_gates():
     np.testing.assert_allclose(oracle.dit_layer(h, lw, m_m2, kp, vp, pos, d), base, rtol=1e-13, atol=1e-14)
     # and each branch does contribute when its gate is on
     assert np.max(np.abs(oracle.dit_layer(h, lw, mod, kp, vp, pos, d) - base)) > 1e-6
+
+
+# ----------------------------------------------------------------- INT8 weights (row-wise)
+
+def test_int8_max_entry_maps_to_127_and_codes_are_bounded():
+    w = RNG.standard_normal((64, 300)).astype(np.float32) * 0.02
+    codes, scales = oracle.quantize_rowwise_int8(w)
+    assert codes.dtype == np.int8 and scales.dtype == np.float32
+    assert codes.min() >= -127 and codes.max() <= 127
+    amax = np.max(np.abs(w), axis=1)
+    np.testing.assert_array_equal(scales, (amax / np.float32(127.0)).astype(np.float32))
+    arg = np.argmax(np.abs(w), axis=1)
+    np.testing.assert_array_equal(np.abs(codes[np.arange(64), arg]), 127)
+    # the dequantisation error of every element is at most half a step
+    err = np.abs(oracle.dequantize_rowwise_int8(codes, scales) - w.astype(np.float64))
+    assert np.all(err <= scales.astype(np.float64)[:, None] * 0.5 * (1 + 1e-6))
+
+
+def test_int8_integer_multiples_round_trip_and_ties_to_even():
+    # scale 1 exactly (row max 127): integers round-trip, halves go to the even neighbour
+    row = np.array([127.0, -127.0, 3.0, -64.0, 0.0, 2.5, 3.5, -2.5, -3.5, 0.5, -0.5, 126.5], np.float32)
+    codes, scales = oracle.quantize_rowwise_int8(row[None, :])
+    assert scales[0] == np.float32(1.0)
+    np.testing.assert_array_equal(codes[0], [127, -127, 3, -64, 0, 2, 4, -2, -4, 0, 0, 126])
+
+
+def test_int8_zero_row_and_torch_round():
+    w = RNG.standard_normal((8, 77)).astype(np.float32)
+    w[3] = 0.0
+    codes, scales = oracle.quantize_rowwise_int8(w)
+    assert scales[3] == 1.0 and not codes[3].any()
+    # torch.round is round-half-to-even on the same fp32 quotients
+    q = torch.from_numpy(w) / torch.from_numpy(scales)[:, None]
+    want = torch.clamp(torch.round(q), -127, 127).to(torch.int8).numpy()
+    np.testing.assert_array_equal(codes, want)
