@@ -93,8 +93,11 @@ __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bflo
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));
 }
 
-template <int EPI, bool FP8, bool NORM>
+// WQ: weight format, 0 bf16 tiles, 1 e4m3 codes, 2 int8 codes (8-bit formats carry one fp32 scale
+// per output row, applied in the epilogue, and are widened to bf16 tiles on chip before the MMA)
+template <int EPI, int WQ, bool NORM>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __grid_constant__ GemmParams p) {
+  constexpr bool FP8 = WQ != 0;   // 8-bit packed weights (e4m3 or int8)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
     const int mtid = threadIdx.x - 64;   // 0..127
     int conv_done = 0;
     auto convert_one = [&](int i) -> bool {
-      // fp8 tile (128 rows x 128 B, swizzled by 16 B chunks) -> two bf16 SW128 tiles
+      // 8-bit tile (128 rows x 128 B, swizzled by 16 B chunks) -> two bf16 SW128 tiles
       const int s = i % p.stages, c = i % kConvStages;
       if (!mbar_wait(&full[s], (i / p.stages) & 1, p.status, DEV_ERR_TIMEOUT_TMA)) return false;
       if (i >= kConvStages && !mbar_wait(&cempty[c], ((i / kConvStages) - 1) & 1, p.status, DEV_ERR_TIMEOUT_CONV))
@@ -277,8 +280,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
         uint32_t o[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          o[2 * q] = e4m3x2_to_bf16x2((uint16_t)(w4[q] & 0xFFFFu));
-          o[2 * q + 1] = e4m3x2_to_bf16x2((uint16_t)(w4[q] >> 16));
+          o[2 * q] = q8x2_to_bf16x2<WQ>((uint16_t)(w4[q] & 0xFFFFu));
+          o[2 * q + 1] = q8x2_to_bf16x2<WQ>((uint16_t)(w4[q] >> 16));
         }
         const int half = ch >> 2;                // which 64-wide bf16 tile
         const int bch = (ch & 3) * 2;            // first bf16 chunk (8 elements) inside it

@@ -226,6 +226,39 @@ __global__ void quant_e4m3_kernel(const __nv_bfloat16* const* __restrict__ rows,
   }
 }
 
+// Row-wise symmetric int8 packing: scale = max|w| / 127 (1 for a zero row), code =
+// round-to-nearest-even(w / scale) clamped to [-127, 127] (code -128 unused), laid out like the
+// e4m3 tiles (128 rows x 128 codes per 16 KB tile, 16-byte chunks swizzled).
+__global__ void quant_int8_kernel(const __nv_bfloat16* const* __restrict__ rows, int K, int Mt, int KB8,
+                                  uint8_t* __restrict__ dst, float* __restrict__ scales) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= Mt * 128) return;
+  const __nv_bfloat16* src = rows[row];
+  float amax = 0.f;
+  if (src)
+    for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(__bfloat162float(src[k])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float sc = amax == 0.f ? 1.f : __fdiv_rn(amax, 127.f);
+  if (lane == 0) scales[row] = sc;
+  const int mt = row >> 7, r = row & 127;
+  for (int c = lane; c < KB8 * 8; c += 32) {            // 16-element chunks along K
+    const int kb = c >> 3, ch = c & 7, k0 = c * 16;
+    uint32_t word[4] = {0, 0, 0, 0};
+    if (src) {
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int k = k0 + q;
+        const float v = k < K ? rintf(__fdiv_rn(__bfloat162float(src[k]), sc)) : 0.f;   // ties to even
+        const int code = max(-127, min(127, (int)v));
+        word[q >> 2] |= (uint32_t)(code & 0xFF) << ((q & 3) * 8);
+      }
+    }
+    *reinterpret_cast<uint4*>(dst + ((size_t)mt * KB8 + kb) * kTileBytesPack + sw128_chunk_byte(r, ch)) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+  }
+}
+
 // ---------------------------------------------------------------- prefix layout (set_prefix)
 // user K, V: [B][L][P][nkv][hd]  ->  K cache [L][B][nkv][Lpad][hd], V^T cache [L][B][nkv][hd][Lpad]
 __global__ void prefix_layout_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -292,10 +325,10 @@ __global__ void untile_kernel(const __nv_bfloat16* tiles, float* out, int Ntok, 
 }
 
 // W . shift for every packed row of one op of one layer and every step:
-// out[k][pr] = sum_c W[pr][c] shift_k[c], with W read back from the packed tiles (fp8: decoded
-// code times the row scale, i.e. exactly the weights the GEMM multiplies).  One warp per row.
+// out[k][pr] = sum_c W[pr][c] shift_k[c], with W read back from the packed tiles (8-bit formats:
+// decoded code times the row scale, i.e. exactly the weights the GEMM multiplies).  One warp per row.
 __global__ void cshift_kernel(const uint8_t* __restrict__ wt, const float* __restrict__ wscale, int rows, int KBt,
-                              int K, int fp8, const float* __restrict__ shift, size_t shift_step_stride, int steps,
+                              int K, int wq, const float* __restrict__ shift, size_t shift_step_stride, int steps,
                               float* out, size_t out_step_stride) {
   const int pr = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (pr >= rows) return;
@@ -305,10 +338,10 @@ __global__ void cshift_kernel(const uint8_t* __restrict__ wt, const float* __res
     const float* sh = shift + (size_t)k * shift_step_stride;
     for (int c = lane; c < K; c += 32) {
       float w;
-      if (fp8) {
+      if (wq) {   // 8-bit codes (1: e4m3, 2: int8) times the row scale
         const uint8_t* tile = wt + ((size_t)mt * KBt + c / 128) * kTileBytesPack;
         const uint8_t code = tile[sw128_chunk_byte(r, (c % 128) / 16) + (c % 16)];
-        const uint32_t pair = e4m3x2_to_bf16x2((uint16_t)code);
+        const uint32_t pair = wq == 2 ? s8x2_to_bf16x2((uint16_t)code) : e4m3x2_to_bf16x2((uint16_t)code);
         w = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(&pair)) * wscale[pr];
       } else {
         const __nv_bfloat16* tile = reinterpret_cast<const __nv_bfloat16*>(wt + ((size_t)mt * KBt + c / 64) * kTileBytesPack);

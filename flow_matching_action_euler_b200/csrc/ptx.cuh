@@ -280,6 +280,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
   __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
   return *reinterpret_cast<uint32_t*>(&b);
 }
+// int8 pair (low byte first) -> bf16x2; exact (every integer of magnitude <= 128 is a bf16 value)
+__device__ __forceinline__ uint32_t s8x2_to_bf16x2(uint16_t two) {
+  const float a = (float)(int8_t)(two & 0xFFu), b = (float)(int8_t)(two >> 8);
+  __nv_bfloat162 r = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+// 8-bit weight pair -> bf16x2 for weight format WQ (1: e4m3, 2: int8)
+template <int WQ>
+__device__ __forceinline__ uint32_t q8x2_to_bf16x2(uint16_t two) {
+  if constexpr (WQ == 2) return s8x2_to_bf16x2(two);
+  else return e4m3x2_to_bf16x2(two);
+}
 // fp32 pair -> e4m3x2, round to nearest even with saturation to +-448 (hardware conversion).
 __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
   uint16_t r;

@@ -76,7 +76,8 @@ struct StepTables {
 struct vla_ae {
   vla_ae_dims d{};
   int device = 0, num_sms = 148;
-  bool fp8 = false;
+  bool fp8 = false;           // 8-bit weight codes with per-row scales (e4m3 or int8)
+  int wq = 0;                 // weight format: 0 bf16, 1 e4m3, 2 int8
   int Ts = 0, Ntok = 0, NT = 0, Nt = 0, qd = 0, kd = 0, Lpad = 0;
   OpPlan op[4];
   size_t layer_wbytes = 0, layer_scales = 0;
@@ -174,11 +175,16 @@ cudaError_t launch_coop(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStr
 
 using GemmKernel = void (*)(const GemmParams);
 
-GemmKernel gemm_kernel_for(OpId id, bool fp8) {
+template <int EPI, bool NORM>
+GemmKernel gemm_kernel_wq(int wq) {
+  return wq == 2 ? gemm_stream_kernel<EPI, 2, NORM> : wq == 1 ? gemm_stream_kernel<EPI, 1, NORM>
+                                                                : gemm_stream_kernel<EPI, 0, NORM>;
+}
+GemmKernel gemm_kernel_for(OpId id, int wq) {
   switch (id) {
-    case OP_QKV: return fp8 ? gemm_stream_kernel<EPI_QKV, true, true> : gemm_stream_kernel<EPI_QKV, false, true>;
-    case OP_GU: return fp8 ? gemm_stream_kernel<EPI_SWIGLU, true, true> : gemm_stream_kernel<EPI_SWIGLU, false, true>;
-    default: return fp8 ? gemm_stream_kernel<EPI_RESID, true, false> : gemm_stream_kernel<EPI_RESID, false, false>;
+    case OP_QKV: return gemm_kernel_wq<EPI_QKV, true>(wq);
+    case OP_GU: return gemm_kernel_wq<EPI_SWIGLU, true>(wq);
+    default: return gemm_kernel_wq<EPI_RESID, false>(wq);
   }
 }
 
@@ -254,7 +260,7 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
   base.KB = ceil_div(K, 64);
   base.KBt = fp8 ? ceil_div(K, 128) : base.KB;
   base.wbytes = (size_t)base.Mt * base.KBt * kTileBytes;
-  GemmKernel kern = gemm_kernel_for(id, fp8);
+  GemmKernel kern = gemm_kernel_for(id, H->wq);
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
   // every kernel of the loop asks for the same (maximum) shared-memory carveout, so SMs never
@@ -349,7 +355,7 @@ int validate_dims(const vla_ae_dims* d) {
   if (d->action_dim > kMaxAction) return VLA_AE_EINVAL;
   if ((long long)d->batch * (d->n_action_tokens + d->has_state_token) > 4096) return VLA_AE_EINVAL;
   if (!(d->rope_theta > 0.f) || !(d->rms_eps >= 0.f)) return VLA_AE_EINVAL;
-  if (d->wtype != VLA_AE_BF16 && d->wtype != VLA_AE_FP8_E4M3) return VLA_AE_EINVAL;
+  if (d->wtype != VLA_AE_BF16 && d->wtype != VLA_AE_FP8_E4M3 && d->wtype != VLA_AE_INT8) return VLA_AE_EINVAL;
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return VLA_AE_EUNSUPPORTED;
   return VLA_AE_OK;
 }
@@ -646,7 +652,7 @@ void set_prefetch(const vla_ae* H, GemmParams& g, OpId id, int layer) {
 
 cudaError_t launch_gemm(const vla_ae* H, OpId id, const GemmParams& g, cudaStream_t st) {
   const OpPlan& p = H->op[id];
-  return launch(gemm_kernel_for(id, H->fp8), dim3(p.S, ceil_div(p.Mt, p.mpc), H->Nt), dim3(kGemmThreads), p.smem, st,
+  return launch(gemm_kernel_for(id, H->wq), dim3(p.S, ceil_div(p.Mt, p.mpc), H->Nt), dim3(kGemmThreads), p.smem, st,
                 p.S, true, g);
 }
 
@@ -941,11 +947,11 @@ int get_tables_grid(vla_ae* H, const std::vector<double>& grid, bool uniform, St
     const size_t mstep = (size_t)d.n_layers * 6 * Hd;
     const OpPlan& pq = H->op[OP_QKV];
     cshift_kernel<<<ceil_div((int)rq, 8), 256, 0, H->cap>>>(wl + pq.woff, sl ? sl + pq.soff : nullptr, (int)rq, pq.KBt,
-                                                           pq.K, H->fp8, mod_l + 0 * Hd, mstep, steps,
+                                                           pq.K, H->wq, mod_l + 0 * Hd, mstep, steps,
                                                            T.cq + (size_t)l * rq, (size_t)d.n_layers * rq);
     const OpPlan& pg = H->op[OP_GU];
     cshift_kernel<<<ceil_div((int)rg, 8), 256, 0, H->cap>>>(wl + pg.woff, sl ? sl + pg.soff : nullptr, (int)rg, pg.KBt,
-                                                           pg.K, H->fp8, mod_l + 3 * Hd, mstep, steps,
+                                                           pg.K, H->wq, mod_l + 3 * Hd, mstep, steps,
                                                            T.cg + (size_t)l * rg, (size_t)d.n_layers * rg);
   }
   CK(cudaGetLastError());
@@ -1033,7 +1039,10 @@ int pack_weights(vla_ae* H, const vla_ae_weights* w) {
       }
       CK(cudaMemcpy(rowptr_dev, rows.data(), (size_t)p.Mt * 128 * sizeof(void*), cudaMemcpyHostToDevice));
       uint8_t* dst = H->wpack + (size_t)l * H->layer_wbytes + p.woff;
-      if (H->fp8) {
+      if (H->wq == 2) {
+        quant_int8_kernel<<<ceil_div(p.Mt * 128, 8), 256>>>(rowptr_dev, p.K, p.Mt, p.KBt, dst,
+                                                           H->wscale + (size_t)l * H->layer_scales + p.soff);
+      } else if (H->wq == 1) {
         quant_e4m3_kernel<<<ceil_div(p.Mt * 128, 8), 256>>>(rowptr_dev, p.K, p.Mt, p.KBt, dst,
                                                            H->wscale + (size_t)l * H->layer_scales + p.soff);
       } else {
@@ -1052,7 +1061,8 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   int rc;
   H->d = *dims;
   const vla_ae_dims& d = H->d;
-  H->fp8 = d.wtype == VLA_AE_FP8_E4M3;
+  H->wq = d.wtype == VLA_AE_FP8_E4M3 ? 1 : d.wtype == VLA_AE_INT8 ? 2 : 0;
+  H->fp8 = H->wq != 0;
   CK(cudaGetDevice(&H->device));
   CK(cudaDeviceGetAttribute(&H->num_sms, cudaDevAttrMultiProcessorCount, H->device));
   int major = 0;

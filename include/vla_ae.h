@@ -40,7 +40,10 @@ extern "C" {
 #define VLA_AE_EUNSUPPORTED (-6) /* valid dims this build does not implement (e.g. head_dim) */
 
 /* ------------------------------------------------------------------ configuration */
-typedef enum { VLA_AE_BF16 = 0, VLA_AE_FP8_E4M3 = 1 } vla_ae_wtype;
+/* Weight formats of the per-layer linears.  FP8_E4M3: the FP8 weights of the APXInf article
+ * (section "CUDA Graph、FP8 和 Rust").  INT8: the INT8 quantisation the same section names for
+ * GPUs without FP8 tensor cores (Jetson Orin), here weight-only with one scale per output channel. */
+typedef enum { VLA_AE_BF16 = 0, VLA_AE_FP8_E4M3 = 1, VLA_AE_INT8 = 2 } vla_ae_wtype;
 
 /* Model and workload dimensions, fixed at create time.
  * Requirements (else VLA_AE_EINVAL): every count >= 1 except has_state_token (0/1) and
@@ -71,9 +74,12 @@ typedef struct {
  * scale).  wq [nq*hd][H], wk/wv [nkv*hd][H], wo [H][nq*hd], wg/wu [I][H], wd [H][I];
  * w_in/w_state [H][A], b_in/b_state [H], w_out [A][H], b_out [A]; w_state/b_state are ignored
  * (may be NULL) without a state token.  on_device: 1 = all pointers are device memory,
- * 0 = host memory; device per-layer matrices must be 16-byte aligned.  With wtype FP8 the library quantises q/k/v/o/gate/up/down itself (one fp32
- * scale per output channel, scale = max|w|/448, codes = e4m3 round-to-nearest-even saturating
- * of w/scale); everything else stays bf16.  The caller keeps ownership; the library copies. */
+ * 0 = host memory; device per-layer matrices must be 16-byte aligned.  With wtype FP8 the
+ * library quantises q/k/v/o/gate/up/down itself (one fp32 scale per output channel, scale =
+ * max|w|/448, codes = e4m3 round-to-nearest-even saturating of w/scale); with wtype INT8 likewise
+ * with scale = max|w|/127 and codes = round-to-nearest-even of w/scale clamped to [-127, 127]
+ * (a zero row takes scale 1); everything else stays bf16.  The caller keeps ownership; the
+ * library copies. */
 typedef struct {
   const void *w_in, *b_in, *w_state, *b_state;
   const void *const *w_ada, *const *b_ada;
@@ -216,8 +222,9 @@ int vla_ae_debug_wait_probe(vla_ae_t h, unsigned attempts);
 int vla_ae_debug_velocity(vla_ae_t h, int step, int steps, const float *x, float *v);
 
 /* Read back one packed per-layer weight in [out][in] order (which: 0 q, 1 k, 2 v, 3 o, 4 gate,
- * 5 up, 6 down) into host memory: bf16 weights as uint16 bits, FP8 weights as e4m3 codes
- * (uint8) plus fp32 scales [out] (scales may be NULL for bf16).  Synchronous. */
+ * 5 up, 6 down) into host memory: bf16 weights as uint16 bits, FP8 / INT8 weights as their
+ * 8-bit codes (e4m3 bits / two's-complement int8) plus fp32 scales [out] (scales may be NULL for
+ * bf16).  Synchronous. */
 int vla_ae_debug_weight(vla_ae_t h, int layer, int which, void *w_host, float *scales_host);
 
 #ifdef __cplusplus

@@ -70,9 +70,9 @@ def test_full_size_bf16(name):
         c.close()
 
 
-@pytest.mark.parametrize("steps", [1, 10])
-def test_full_size_fp8(steps):
-    c = Case(config("pi05_fp8", steps=steps))
+@pytest.mark.parametrize("wtype,steps", [("pi05_fp8", 1), ("pi05_fp8", 10), ("pi05_int8", 1), ("pi05_int8", 10)])
+def test_full_size_fp8(wtype, steps):
+    c = Case(config(wtype, steps=steps))
     try:
         got = c.denoise()
         ref_q = c.oracle_denoise()

@@ -96,6 +96,19 @@ def test_fp8_codes_and_scales_bitexact():
             assert np.array_equal(got, codes), (layer, key, int(np.sum(got != codes)))
 
 
+def test_int8_codes_and_scales_bitexact():
+    c = case("ragged", wtype="int8")
+    for layer in range(c.d.n_layers):
+        for which, key in enumerate(("wq", "wk", "wv", "wo", "wg", "wu", "wd")):
+            w32 = oracle.bf16_to_f64(c.w["layers"][layer][key]).astype(np.float32)
+            codes, scales = oracle.quantize_rowwise_int8(w32)
+            got = np.zeros(codes.shape, np.uint8)
+            gs = np.zeros(scales.shape, np.float32)
+            c.ae.debug_weight(layer, which, got, gs)
+            assert np.array_equal(gs.view(np.uint32), scales.view(np.uint32)), (layer, key)
+            assert np.array_equal(got.view(np.int8), codes), (layer, key, int(np.sum(got.view(np.int8) != codes)))
+
+
 # ------------------------------------------------------------------ one layer, teacher-forced
 
 def _layer_check(c, step, steps, layers=None, tol=LAYER_TOL):
@@ -297,6 +310,17 @@ def test_fp8_tiny():
     ref_bf16 = c.oracle_denoise(W=oracle.OracleWeights(c.w, c.d, quantized=False))
     assert rel_err(got, ref_q) <= 2e-2
     assert rel_err(got, ref_bf16) <= FP8_TOL
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_int8(name):
+    c = case(name, wtype="int8")
+    got = c.denoise()
+    ref_q = c.oracle_denoise()
+    ref_bf16 = c.oracle_denoise(W=oracle.OracleWeights(c.w, c.d, quantized=False))
+    assert rel_err(got, ref_q) <= 2e-2
+    assert rel_err(got, ref_bf16) <= FP8_TOL
+    _layer_check(c, 0, c.d.steps, layers=[0])
 
 
 def test_bounded_wait_reports_timeout_and_handle_stays_usable():
