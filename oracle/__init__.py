@@ -18,6 +18,8 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
                        skipped-step grid equals a brute-force velocity cache
                        (DP-Cache reading); first-order convergence on a graded
                        grid; the one-step grid; grid validation
+``euler_integrate_switch`` closed form for two linear fields (matrix powers),
+                       n_stale = 0 / N reduce to one field
 ``timestep_embedding`` t = 0 gives [1..1, 0..0]; first frequency is 1000 t;
                        last frequency matches the base-10000 geometric series
 ``rms_norm``           unit RMS at eps = 0, scale invariance, torch's rms_norm
@@ -41,7 +43,7 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
 from .model import (  # noqa: F401
     bf16_to_f64, t_schedule, timestep_embedding, silu, rms_norm, modulate, rope_half,
     rope_positions_angles, gqa_attention, linear, swiglu, euler_integrate, euler_integrate_grid,
-    check_t_grid, uniform_grid,
+    check_t_grid, uniform_grid, euler_integrate_switch, denoise_stale,
     adaln_table, dit_layer, embed_tokens, velocity, denoise, denoise_batch, OracleWeights,
 )
 from .fp8 import (  # noqa: F401

@@ -78,6 +78,21 @@ def euler_integrate_grid(x0: np.ndarray, t_grid, v_fn: Callable[[np.ndarray, flo
     return x
 
 
+def euler_integrate_switch(x0: np.ndarray, n_steps: int, n_stale: int,
+                           v_before: Callable[[np.ndarray, float], np.ndarray],
+                           v_after: Callable[[np.ndarray, float], np.ndarray]) -> np.ndarray:
+    """Fixed-step Euler whose field changes after ``n_stale`` steps ("跨XPU平台表征视觉-语言-动作模型"
+    section 5.3, V-AEFusion: the first steps reuse the previous cycle's visual features):
+    x_{k+1} = x_k + dt * v_before(x_k, t_k) for k < n_stale, then v_after."""
+    if not 0 <= n_stale <= n_steps:
+        raise ValueError("0 <= n_stale <= n_steps")
+    ts, dt = t_schedule(n_steps)
+    x = np.array(x0, dtype=np.float64, copy=True)
+    for k, t in enumerate(ts):
+        x = x + dt * (v_before if k < n_stale else v_after)(x, t)
+    return x
+
+
 def euler_integrate(x0: np.ndarray, n_steps: int, v_fn: Callable[[np.ndarray, float], np.ndarray]) -> np.ndarray:
     """Fixed-step explicit Euler from t = 1 to t = 0: x_{k+1} = x_k + dt * v(x_k, t_k)."""
     ts, dt = t_schedule(n_steps)
@@ -283,6 +298,15 @@ def denoise(noise: np.ndarray, state: Optional[np.ndarray], W: OracleWeights, k_
     if t_grid is not None:
         return euler_integrate_grid(noise, t_grid, v_fn)
     return euler_integrate(noise, n_steps, v_fn)
+
+
+def denoise_stale(noise: np.ndarray, before, after, W: OracleWeights, d, n_steps: int, n_stale: int) -> np.ndarray:
+    """x_N of the N-step loop whose first ``n_stale`` steps see prefix ``before`` and the rest
+    ``after``; each prefix is (state, k_prefix, v_prefix) in float64 (state None without a state
+    token)."""
+    vb = lambda x, t: velocity(x, t, before[0], W, before[1], before[2], d)
+    va = lambda x, t: velocity(x, t, after[0], W, after[1], after[2], d)
+    return euler_integrate_switch(noise, n_steps, n_stale, vb, va)
 
 
 def denoise_batch(weights_bits: Dict[str, object], inputs_bits: Dict[str, np.ndarray], d,

@@ -150,6 +150,32 @@ def test_euler_grid_rejects_bad_grids(grid):
         oracle.check_t_grid(grid)
 
 
+# ----------------------------------------------------------------- Euler with a switched field
+
+@pytest.mark.parametrize("n_steps,n_stale", [(4, 2), (10, 5), (7, 1), (7, 6)])
+def test_euler_switch_linear_fields_closed_form(n_steps, n_stale):
+    a1, b1, x0 = _linear_field(seed=11)
+    a2, b2, _ = _linear_field(seed=12)
+    got = oracle.euler_integrate_switch(x0, n_steps, n_stale, lambda x, t: a1 @ x + b1, lambda x, t: a2 @ x + b2)
+    dt = -1.0 / n_steps
+    m1, m2 = np.eye(7) + dt * a1, np.eye(7) + dt * a2
+    mp = np.linalg.matrix_power
+    xs = mp(m1, n_stale) @ x0 + sum((mp(m1, j) @ (dt * b1) for j in range(n_stale)), np.zeros(7))
+    want = mp(m2, n_steps - n_stale) @ xs + sum((mp(m2, j) @ (dt * b2) for j in range(n_steps - n_stale)), np.zeros(7))
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_euler_switch_extremes_reduce_to_one_field():
+    a1, b1, x0 = _linear_field(seed=13)
+    f1 = lambda x, t: np.tanh(a1 @ x) + t
+    f2 = lambda x, t: np.sin(x) - b1
+    for n in (1, 4):
+        assert np.array_equal(oracle.euler_integrate_switch(x0, n, n, f1, f2), oracle.euler_integrate(x0, n, f1))
+        assert np.array_equal(oracle.euler_integrate_switch(x0, n, 0, f1, f2), oracle.euler_integrate(x0, n, f2))
+    with pytest.raises(ValueError):
+        oracle.euler_integrate_switch(x0, 4, 5, f1, f2)
+
+
 # ----------------------------------------------------------------- time embedding
 
 def test_timestep_embedding_t0_and_identity():
