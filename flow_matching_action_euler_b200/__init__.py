@@ -17,7 +17,7 @@ __all__ = [
     "lib", "VlaAeDims", "VlaAeWeights", "VlaAeTrace", "VlaAeError", "ActionExpert",
     "vla_ae_create", "vla_ae_set_prefix", "vla_ae_denoise", "vla_ae_denoise_host", "vla_ae_status",
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
-    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "vla_ae_denoise_sched", "BF16", "FP8_E4M3", "INT8", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
+    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "vla_ae_denoise_sched", "vla_ae_set_prefix_next", "vla_ae_denoise_stale", "BF16", "FP8_E4M3", "INT8", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
     "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES", "Q_ENGINE", "ENGINE_PER_OP", "ENGINE_PERSISTENT",
 ]
 
@@ -80,6 +80,8 @@ vla_ae_debug_weight = _sig("vla_ae_debug_weight", ctypes.c_int, _H, ctypes.c_int
 vla_ae_bench_op = _sig("vla_ae_bench_op", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P)
 vla_ae_debug_wait_probe = _sig("vla_ae_debug_wait_probe", ctypes.c_int, _H, ctypes.c_uint)
 vla_ae_set_engine = _sig("vla_ae_set_engine", ctypes.c_int, _H, ctypes.c_int)
+vla_ae_set_prefix_next = _sig("vla_ae_set_prefix_next", ctypes.c_int, _H, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P)
+vla_ae_denoise_stale = _sig("vla_ae_denoise_stale", ctypes.c_int, _H, _P, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_denoise_sched = _sig("vla_ae_denoise_sched", ctypes.c_int, _H, _P, ctypes.POINTER(ctypes.c_float),
                             ctypes.c_int, _P, _P)
 vla_ae_set_prefix_static = _sig("vla_ae_set_prefix_static", ctypes.c_int, _H, _P, _P, ctypes.c_int, _P, _P)
@@ -160,6 +162,16 @@ class ActionExpert:
     def denoise(self, noise, steps: int, out, stream=None):
         _check(vla_ae_denoise(self.handle, _ptr(noise), int(steps), _ptr(out), _stream_ptr(stream)),
                "vla_ae_denoise")
+
+    def set_prefix_next(self, k, v, n_prefix: int, state=None, on_device: bool = False, stream=None):
+        """Lay out the next cycle's prefix (see vla_ae_set_prefix_next)."""
+        _check(vla_ae_set_prefix_next(self.handle, _ptr(k), _ptr(v), int(n_prefix), _ptr(state), int(on_device),
+                                      _stream_ptr(stream)), "vla_ae_set_prefix_next")
+
+    def denoise_stale(self, noise, steps: int, n_stale: int, out, stream=None):
+        """Steps [0, n_stale) on the current prefix, the rest on the next one (see vla_ae_denoise_stale)."""
+        _check(vla_ae_denoise_stale(self.handle, _ptr(noise), int(steps), int(n_stale), _ptr(out),
+                                    _stream_ptr(stream)), "vla_ae_denoise_stale")
 
     def denoise_sched(self, noise, t_grid: Sequence[float], out, stream=None):
         """Euler along the time grid t_grid[0] > ... > t_grid[n] (n steps)."""

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -66,9 +67,16 @@ struct StepTables {
   unsigned* ctr = nullptr;  // persistent engine: per-step counter blocks [steps][ctr_step]
   std::vector<double> t;    // time grid t_0 > ... > t_steps
   std::vector<float> dt;    // Euler step k: t_{k+1} - t_k
-  cudaGraphExec_t exec = nullptr;
-  int captured_prefix = -1;
-  int captured_engine = -1;
+  // captured graphs, one per (first step, end step, prefix slot, prefix length, engine)
+  std::map<std::array<int, 5>, cudaGraphExec_t> graphs;
+};
+
+// One prefix buffer set: the layer caches (prefix rows + the self rows the loop writes), the
+// RoPE table of the self-token positions and the projected state token.
+struct PrefixSlot {
+  __nv_bfloat16 *kc = nullptr, *vct = nullptr;
+  float *rope = nullptr, *h_state0 = nullptr;
+  int n_prefix = -1;
 };
 
 }  // namespace
@@ -104,6 +112,13 @@ struct vla_ae {
   unsigned* status = nullptr;
   size_t device_bytes = 0;
   int n_prefix = -1;
+  // prefix slots: slot[front] is the one the loop reads (mirrored in kc / vct / rope / h_state0 /
+  // n_prefix above); the other is the back slot vla_ae_set_prefix_next fills
+  PrefixSlot slot[2];
+  int front = 0;
+  bool next_pending = false;
+  cudaEvent_t next_ready = nullptr;
+  int attn_P = -1;            // prefix length the per-op attention plan was made for
   cudaStream_t cap = nullptr;
   std::map<std::vector<double>, StepTables> tables;   // keyed by the time grid
 
@@ -120,7 +135,8 @@ struct vla_ae {
   }
   ~vla_ae() {
     for (auto& kv : tables)
-      if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+      for (auto& g : kv.second.graphs) cudaGraphExecDestroy(g.second);
+    if (next_ready) cudaEventDestroy(next_ready);
     for (void* p : allocs) cudaFree(p);
     if (cap) cudaStreamDestroy(cap);
   }
@@ -849,49 +865,34 @@ cudaError_t launch_loop(const vla_ae* H, const StepTables& T, int step, unsigned
                      st, lp);
 }
 
-cudaError_t enqueue_loop(vla_ae* H, const StepTables& T, cudaStream_t st) {
+// Euler steps [k0, k1) of the loop of T.  The first step of the loop starts from the noise; a
+// later segment starts from x as the previous segment left it (its in-projection runs here, so
+// a segment uses its own prefix slot's state token).  The last step writes the actions.
+cudaError_t enqueue_steps(vla_ae* H, const StepTables& T, int k0, int k1, cudaStream_t st) {
   const int N = T.steps, L = H->d.n_layers;
-  if (H->use_loop) {
-    cudaError_t e = cudaMemsetAsync(T.ctr, 0, (size_t)N * H->ctr_step * 4, st);
-    if (e != cudaSuccess) return e;
-    TailParams t0 = tail_common(H);
-    t0.init_from_noise = 1;
-    t0.do_in = 1;
-    t0.sc_next = layer_mod(H, T, 0, 0).scale_a;
-    if ((e = launch_tail(H, t0, st)) != cudaSuccess) return e;
-    for (int k = 0; k < N; ++k) {
-      if ((e = launch_loop(H, T, k, T.ctr + (size_t)k * H->ctr_step, 0, 0, L, kPhases, 1, st)) != cudaSuccess) return e;
-      TailParams t = tail_common(H);
-      t.ss_parts = ss_parts_final(H);
-      t.shift_f = T.fmod + (size_t)k * 2 * H->d.hidden;
-      t.scale_f = t.shift_f + H->d.hidden;
-      t.dt = T.dt[k];
-      t.do_out = 1;
-      t.do_in = k + 1 < N;
-      if (t.do_in) t.sc_next = layer_mod(H, T, k + 1, 0).scale_a;
-      t.out = k + 1 == N ? H->out_stage : nullptr;
-      if ((e = launch_tail(H, t, st)) != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-  }
-  TailParams t0 = tail_common(H);
-  t0.init_from_noise = 1;
-  t0.do_in = 1;
-  t0.sc_next = layer_mod(H, T, 0, 0).scale_a;
   cudaError_t e;
+  if (H->use_loop && (e = cudaMemsetAsync(T.ctr + (size_t)k0 * H->ctr_step, 0,
+                                          (size_t)(k1 - k0) * H->ctr_step * 4, st)) != cudaSuccess)
+    return e;
+  TailParams t0 = tail_common(H);
+  t0.init_from_noise = k0 == 0;
+  t0.do_in = 1;
+  t0.sc_next = layer_mod(H, T, k0, 0).scale_a;
   if ((e = launch_tail(H, t0, st)) != cudaSuccess) return e;
-  for (int k = 0; k < N; ++k) {
-    for (int l = 0; l < L; ++l) {
-      const int parts = l == 0 ? 1 : ss_parts_of(H, OP_D);
-      if ((e = enqueue_layer(H, T, k, l, parts, st, nullptr)) != cudaSuccess) return e;
+  for (int k = k0; k < k1; ++k) {
+    if (H->use_loop) {
+      if ((e = launch_loop(H, T, k, T.ctr + (size_t)k * H->ctr_step, 0, 0, L, kPhases, 1, st)) != cudaSuccess) return e;
+    } else {
+      for (int l = 0; l < L; ++l)
+        if ((e = enqueue_layer(H, T, k, l, l == 0 ? 1 : ss_parts_of(H, OP_D), st, nullptr)) != cudaSuccess) return e;
     }
     TailParams t = tail_common(H);
-    t.ss_parts = ss_parts_of(H, OP_D);
+    t.ss_parts = ss_parts_final(H);
     t.shift_f = T.fmod + (size_t)k * 2 * H->d.hidden;
     t.scale_f = t.shift_f + H->d.hidden;
     t.dt = T.dt[k];
     t.do_out = 1;
-    t.do_in = k + 1 < N;
+    t.do_in = k + 1 < k1;
     if (t.do_in) t.sc_next = layer_mod(H, T, k + 1, 0).scale_a;
     t.out = k + 1 == N ? H->out_stage : nullptr;
     if ((e = launch_tail(H, t, st)) != cudaSuccess) return e;
@@ -971,26 +972,54 @@ std::vector<double> uniform_grid(int steps) {
 
 int get_tables(vla_ae* H, int steps, StepTables** out) { return get_tables_grid(H, uniform_grid(steps), true, out); }
 
-int ensure_graph(vla_ae* H, StepTables* T) {
-  if (T->exec && T->captured_prefix == H->n_prefix && T->captured_engine == (int)H->use_loop) return VLA_AE_OK;
-  if (T->exec) {
-    cudaGraphExecDestroy(T->exec);
-    T->exec = nullptr;
+// Make prefix slot i the one the loop reads (the kernels take the mirrored fields), re-planning
+// the per-op attention for its prefix length.
+int use_slot(vla_ae* H, int i) {
+  const PrefixSlot& sl = H->slot[i];
+  H->kc = sl.kc;
+  H->vct = sl.vct;
+  H->rope = sl.rope;
+  H->h_state0 = sl.h_state0;
+  H->n_prefix = sl.n_prefix;
+  if (sl.n_prefix >= 0 && sl.n_prefix != H->attn_P) {
+    int rc = plan_attention(H, sl.n_prefix);
+    if (rc) return rc;
+    H->attn_P = sl.n_prefix;
   }
+  return VLA_AE_OK;
+}
+
+// The graph of steps [k0, k1) of T on prefix slot `sl` (captured on first use).
+int ensure_graph(vla_ae* H, StepTables* T, int k0, int k1, int sl, cudaGraphExec_t* out) {
+  const std::array<int, 5> key = {k0, k1, sl, H->slot[sl].n_prefix, (int)H->use_loop};
+  auto it = T->graphs.find(key);
+  if (it != T->graphs.end()) {
+    *out = it->second;
+    return VLA_AE_OK;
+  }
+  int rc = use_slot(H, sl);
+  if (rc) return rc;
   cudaGraph_t g = nullptr;
-  CK(cudaStreamBeginCapture(H->cap, cudaStreamCaptureModeThreadLocal));
-  cudaError_t e = enqueue_loop(H, *T, H->cap);
-  cudaError_t e2 = cudaStreamEndCapture(H->cap, &g);
+  cudaError_t e0 = cudaStreamBeginCapture(H->cap, cudaStreamCaptureModeThreadLocal);
+  cudaError_t e = e0 == cudaSuccess ? enqueue_steps(H, *T, k0, k1, H->cap) : e0;
+  cudaError_t e2 = e0 == cudaSuccess ? cudaStreamEndCapture(H->cap, &g) : e0;
+  rc = use_slot(H, H->front);
   if (e != cudaSuccess || e2 != cudaSuccess) {
     std::fprintf(stderr, "vla_ae: graph capture failed: %s / %s\n", cudaGetErrorString(e), cudaGetErrorString(e2));
     if (g) cudaGraphDestroy(g);
     cudaGetLastError();
     return VLA_AE_ECUDA;
   }
-  CK(cudaGraphInstantiate(&T->exec, g, 0));
+  if (rc) {
+    cudaGraphDestroy(g);
+    return rc;
+  }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t ei = cudaGraphInstantiate(&exec, g, 0);
   cudaGraphDestroy(g);
-  T->captured_prefix = H->n_prefix;
-  T->captured_engine = (int)H->use_loop;
+  CK(ei);
+  T->graphs.emplace(key, exec);
+  *out = exec;
   return VLA_AE_OK;
 }
 
@@ -1116,6 +1145,12 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   if ((rc = H->alloc(&H->out_stage, B * d.n_action_tokens * A * 4))) return rc;
   if ((rc = H->alloc(&H->h_state0, B * Hd * 4))) return rc;
   if ((rc = H->alloc(&H->rope, (size_t)H->Ts * (d.head_dim / 2) * 8))) return rc;
+  H->slot[0].kc = H->kc;
+  H->slot[0].vct = H->vct;
+  H->slot[0].rope = H->rope;
+  H->slot[0].h_state0 = H->h_state0;
+  H->attn_P = d.max_prefix;   // plan_attention ran for max_prefix above
+  CK(cudaEventCreateWithFlags(&H->next_ready, cudaEventDisableTiming));
 
   if (!w) return VLA_AE_EINVAL;
   const int od = w->on_device;
@@ -1186,17 +1221,12 @@ void vla_ae_destroy(vla_ae_t h) {
   delete h;
 }
 
-int vla_ae_set_prefix(vla_ae_t H, const void* k, const void* v, int n_prefix, const void* state, int on_device,
-                      void* stream) {
-  if (!H || n_prefix < 0 || n_prefix > H->d.max_prefix) return VLA_AE_EINVAL;
-  if (n_prefix > 0 && (!k || !v)) return VLA_AE_EINVAL;
-  if (H->d.has_state_token && !state) return VLA_AE_EINVAL;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+// Lay a prefix out into slot i: K / V^T caches, projected state token, RoPE table of the self
+// tokens at positions n_prefix + j.  Asynchronous on st.
+static int write_prefix(vla_ae_t H, int i, const void* k, const void* v, int n_prefix, const void* state,
+                        int on_device, cudaStream_t st) {
   const vla_ae_dims& d = H->d;
-  if (n_prefix != H->n_prefix) {
-    int rc = plan_attention(H, n_prefix);
-    if (rc) return rc;
-  }
+  PrefixSlot& sl = H->slot[i];
   const size_t n = (size_t)d.batch * d.n_layers * n_prefix * d.n_kv_heads * d.head_dim;
   if (n > 0) {
     const __nv_bfloat16 *kd = reinterpret_cast<const __nv_bfloat16*>(k), *vd = reinterpret_cast<const __nv_bfloat16*>(v);
@@ -1209,7 +1239,7 @@ int vla_ae_set_prefix(vla_ae_t H, const void* k, const void* v, int n_prefix, co
       kd = kt;
       vd = vt;
     }
-    prefix_layout_kernel<<<4 * H->num_sms, 256, 0, st>>>(kd, vd, H->kc, H->vct, d.batch, d.n_layers, n_prefix,
+    prefix_layout_kernel<<<4 * H->num_sms, 256, 0, st>>>(kd, vd, sl.kc, sl.vct, d.batch, d.n_layers, n_prefix,
                                                          d.n_kv_heads, d.head_dim, H->Lpad);
     CK(cudaGetLastError());
     if (kt) CK(cudaFreeAsync(kt, st));
@@ -1219,23 +1249,58 @@ int vla_ae_set_prefix(vla_ae_t H, const void* k, const void* v, int n_prefix, co
     CK(cudaMemcpyAsync(H->state_stage, state, (size_t)d.batch * d.action_dim * 2,
                        on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, st));
     state_proj_kernel<<<dim3(ceil_div(d.hidden, 256), d.batch), 256, 0, st>>>(H->w_st, H->b_st, H->state_stage,
-                                                                               H->h_state0, d.hidden, d.action_dim);
+                                                                               sl.h_state0, d.hidden, d.action_dim);
   }
-  rope_table_kernel<<<ceil_div(H->Ts * d.head_dim / 2, 256), 256, 0, st>>>(reinterpret_cast<float2*>(H->rope), H->Ts,
+  rope_table_kernel<<<ceil_div(H->Ts * d.head_dim / 2, 256), 256, 0, st>>>(reinterpret_cast<float2*>(sl.rope), H->Ts,
                                                                            n_prefix, d.head_dim, (double)d.rope_theta);
   CK(cudaGetLastError());
-  H->n_prefix = n_prefix;
+  sl.n_prefix = n_prefix;
+  return VLA_AE_OK;
+}
+
+int vla_ae_set_prefix(vla_ae_t H, const void* k, const void* v, int n_prefix, const void* state, int on_device,
+                      void* stream) {
+  if (!H || n_prefix < 0 || n_prefix > H->d.max_prefix) return VLA_AE_EINVAL;
+  if (n_prefix > 0 && (!k || !v)) return VLA_AE_EINVAL;
+  if (H->d.has_state_token && !state) return VLA_AE_EINVAL;
+  int rc = write_prefix(H, H->front, k, v, n_prefix, state, on_device, reinterpret_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  return use_slot(H, H->front);
+}
+
+int vla_ae_set_prefix_next(vla_ae_t H, const void* k, const void* v, int n_prefix, const void* state, int on_device,
+                           void* stream) {
+  if (!H || n_prefix < 0 || n_prefix > H->d.max_prefix) return VLA_AE_EINVAL;
+  if (n_prefix > 0 && (!k || !v)) return VLA_AE_EINVAL;
+  if (H->d.has_state_token && !state) return VLA_AE_EINVAL;
+  const int back = 1 - H->front;
+  PrefixSlot& sl = H->slot[back];
+  if (!sl.kc) {   // the back slot's buffers, on first use
+    const vla_ae_dims& d = H->d;
+    const size_t cache = (size_t)d.n_layers * d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+    int rc;
+    if ((rc = H->alloc(&sl.kc, cache * 2))) return rc;
+    if ((rc = H->alloc(&sl.vct, cache * 2))) return rc;
+    if ((rc = H->alloc(&sl.h_state0, (size_t)d.batch * d.hidden * 4))) return rc;
+    if ((rc = H->alloc(&sl.rope, (size_t)H->Ts * (d.head_dim / 2) * 8))) return rc;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int rc = write_prefix(H, back, k, v, n_prefix, state, on_device, st);
+  if (rc) return rc;
+  CK(cudaEventRecord(H->next_ready, st));
+  H->next_pending = true;
   return VLA_AE_OK;
 }
 
 static int denoise_tables(vla_ae_t H, StepTables* T, const void* noise, float* out, void* stream, bool host) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaGraphExec_t exec = nullptr;
   int rc;
-  if ((rc = ensure_graph(H, T))) return rc;
+  if ((rc = ensure_graph(H, T, 0, T->steps, H->front, &exec))) return rc;
   const vla_ae_dims& d = H->d;
   const size_t nx = (size_t)d.batch * d.n_action_tokens * d.action_dim;
   CK(cudaMemcpyAsync(H->noise_stage, noise, nx * 2, host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
-  CK(cudaGraphLaunch(T->exec, st));
+  CK(cudaGraphLaunch(exec, st));
   CK(cudaMemcpyAsync(out, H->out_stage, nx * 4, host ? cudaMemcpyDeviceToHost : cudaMemcpyDeviceToDevice, st));
   return VLA_AE_OK;
 }
@@ -1255,6 +1320,29 @@ int vla_ae_denoise(vla_ae_t H, const void* noise, int steps, float* out, void* s
 
 int vla_ae_denoise_host(vla_ae_t H, const void* noise_host, int steps, float* out_host, void* stream) {
   return denoise_common(H, noise_host, steps, out_host, stream, true);
+}
+
+int vla_ae_denoise_stale(vla_ae_t H, const void* noise, int steps, int n_stale, float* out, void* stream) {
+  if (!H || !noise || !out || steps < 1 || n_stale < 0 || n_stale > steps) return VLA_AE_EINVAL;
+  if (H->n_prefix < 0 || !H->next_pending) return VLA_AE_ENOPREFIX;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  StepTables* T = nullptr;
+  int rc = get_tables(H, steps, &T);
+  if (rc) return rc;
+  const int back = 1 - H->front;
+  cudaGraphExec_t ga = nullptr, gb = nullptr;
+  if (n_stale > 0 && (rc = ensure_graph(H, T, 0, n_stale, H->front, &ga))) return rc;
+  if (n_stale < steps && (rc = ensure_graph(H, T, n_stale, steps, back, &gb))) return rc;
+  const vla_ae_dims& d = H->d;
+  const size_t nx = (size_t)d.batch * d.n_action_tokens * d.action_dim;
+  CK(cudaMemcpyAsync(H->noise_stage, noise, nx * 2, cudaMemcpyDeviceToDevice, st));
+  if (ga) CK(cudaGraphLaunch(ga, st));
+  CK(cudaStreamWaitEvent(st, H->next_ready, 0));   // the next prefix is laid out
+  if (gb) CK(cudaGraphLaunch(gb, st));
+  CK(cudaMemcpyAsync(out, H->out_stage, nx * 4, cudaMemcpyDeviceToDevice, st));
+  H->front = back;   // the new prefix is the current one from now on
+  H->next_pending = false;
+  return use_slot(H, H->front);
 }
 
 int vla_ae_denoise_sched(vla_ae_t H, const void* noise, const float* t_grid, int n, float* out, void* stream) {
@@ -1538,10 +1626,6 @@ extern "C" int vla_ae_set_prefix_static(vla_ae_t H, const void* k, const void* v
   int rc = static_scratch(H->device, &scratch);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (n_prefix != H->n_prefix) {
-    rc = plan_attention(H, n_prefix);
-    if (rc) return rc;
-  }
   __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(scratch);
   __nv_bfloat16* vs = ks + (size_t)d.batch * per_sample;
   const size_t cache_layer = (size_t)d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
@@ -1566,6 +1650,6 @@ extern "C" int vla_ae_set_prefix_static(vla_ae_t H, const void* k, const void* v
   rope_table_kernel<<<ceil_div(H->Ts * d.head_dim / 2, 256), 256, 0, st>>>(reinterpret_cast<float2*>(H->rope), H->Ts,
                                                                            n_prefix, d.head_dim, (double)d.rope_theta);
   CK(cudaGetLastError());
-  H->n_prefix = n_prefix;
-  return VLA_AE_OK;
+  H->slot[H->front].n_prefix = n_prefix;   // (H->kc ... mirror the front slot's buffers)
+  return use_slot(H, H->front);
 }

@@ -134,6 +134,27 @@ int vla_ae_set_prefix_static(vla_ae_t h, const void *k, const void *v, int n_pre
  * `stream`.  Errors: EINVAL, ENOPREFIX, ECUDA. */
 int vla_ae_denoise(vla_ae_t h, const void *noise, int steps, float *out, void *stream);
 
+/* ------------------------------------------------------------------ stale-prefix overlap
+ * V-AEFusion ("跨XPU平台表征视觉-语言-动作模型" section 5.3): the first denoising steps of a control
+ * cycle run on the previous cycle's prefix while the VLM computes the new one on another stream;
+ * the remaining steps use the new prefix.
+ *
+ * vla_ae_set_prefix_next: lay out the NEXT cycle's prefix (arguments as vla_ae_set_prefix) into a
+ * second set of caches, asynchronously on `stream` (typically the stream that produced it), and
+ * record a library-owned event there.  The first call allocates that second set.
+ *
+ * vla_ae_denoise_stale: run steps [0, n_stale) of the `steps`-step loop on the current prefix,
+ * make `stream` wait for the event of the last vla_ae_set_prefix_next, run steps [n_stale, steps)
+ * on the next prefix (its state token included), then make the next prefix the current one.
+ * 0 <= n_stale <= steps (0: all steps on the new prefix; steps: all on the old one).  Enqueue
+ * vla_ae_set_prefix_next before this call (both are asynchronous: the overlap happens on the
+ * GPU).  The first call per (steps, n_stale) captures two graphs.
+ * Errors: EINVAL, ENOPREFIX (no current prefix, or no vla_ae_set_prefix_next since the last
+ * vla_ae_denoise_stale), ECUDA. */
+int vla_ae_set_prefix_next(vla_ae_t h, const void *k, const void *v, int n_prefix, const void *state, int on_device,
+                           void *stream);
+int vla_ae_denoise_stale(vla_ae_t h, const void *noise, int steps, int n_stale, float *out, void *stream);
+
 /* The Euler loop along a caller-chosen time grid: n steps x_{k+1} = x_k + (t_{k+1} - t_k) *
  * v(x_k, t_k) for the host array t_grid[0..n] (strictly decreasing, finite; 1 <= n <=
  * VLA_AE_MAX_GRID_STEPS).  It serves step skipping ("跨XPU平台表征视觉-语言-动作模型" sections 5.2

@@ -101,6 +101,8 @@ def test_null_arguments(fm):
     g = (ctypes.c_float * 3)(1.0, 0.5, 0.0)
     assert fm.vla_ae_denoise_sched(None, None, g, 2, None, None) == fm.EINVAL
     assert fm.vla_ae_set_engine(None, fm.ENGINE_PER_OP) == fm.EINVAL
+    assert fm.vla_ae_set_prefix_next(None, None, None, 0, None, 0, None) == fm.EINVAL
+    assert fm.vla_ae_denoise_stale(None, None, 4, 2, None, None) == fm.EINVAL
     fm.vla_ae_destroy(None)   # no-op
 
 

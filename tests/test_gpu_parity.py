@@ -248,6 +248,44 @@ def test_denoise_time_grid_rejects_bad_grids():
         assert e.value.code == fm.EINVAL
 
 
+@pytest.mark.parametrize("eng", ENGINES)
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_stale_prefix_overlap(name, eng):
+    """First n_stale steps on the previous prefix, the rest on the next one; then it is current."""
+    from synth import generate_inputs
+    c = case(name, n_prefix=17, max_prefix=48)
+    d = c.d
+    new = generate_inputs(d, seed=5, n_prefix=48)
+    cur = (c.x.get("state"), c.x["k"], c.x["v"], 17)
+    nxt = (new.get("state"), new["k"], new["v"], 48)
+
+    def pre(p, b):
+        st = oracle.bf16_to_f64(p[0][b]) if d.has_state_token else None
+        return (st, oracle.bf16_to_f64(p[1][b]), oracle.bf16_to_f64(p[2][b]))
+
+    noise = torch.from_numpy(c.x["noise"].view(np.int16)).cuda()
+    out = torch.empty((d.batch, d.n_action_tokens, d.action_dim), dtype=torch.float32, device="cuda")
+    side = torch.cuda.Stream()
+    with engine(c, eng):
+        for n_stale in (0, 2, d.steps):
+            c.ae.set_prefix(cur[1], cur[2], cur[3], cur[0])
+            with torch.cuda.stream(side):   # the "VLM" stream
+                c.ae.set_prefix_next(nxt[1], nxt[2], nxt[3], nxt[0], stream=side)
+            c.ae.denoise_stale(noise, d.steps, n_stale, out)
+            torch.cuda.synchronize()
+            assert c.ae.status() == 0
+            ref = np.stack([oracle.denoise_stale(oracle.bf16_to_f64(c.x["noise"][b]), pre(cur, b), pre(nxt, b),
+                                                 c.W, d, d.steps, n_stale) for b in range(d.batch)])
+            assert rel_err(out.cpu().numpy(), ref) <= FINAL_TOL, n_stale
+            # the next prefix is now the current one
+            ref_new = oracle.denoise_batch(c.w, {**c.x, "k": new["k"], "v": new["v"], "state": new.get("state")}, d,
+                                           W=c.W)
+            assert rel_err(c.denoise(), ref_new) <= FINAL_TOL
+        with pytest.raises(Exception):   # no next prefix since the last stale call
+            c.ae.denoise_stale(noise, d.steps, 1, out)
+        c.ae.set_prefix(cur[1], cur[2], cur[3], cur[0])   # leave the shared case as it was
+
+
 def test_denoise_is_deterministic_across_replays():
     c = case("tiny")
     a = c.denoise()
