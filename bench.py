@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200, help="timed denoise loops")
     ap.add_argument("--warmup", type=int, default=20, help="untimed denoise loops (>= 3)")
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
-    ap.add_argument("--workload", default="starvla", choices=("starvla", "pi05", "pi05_fp8", "pi05_int8", "tiny"))
+    ap.add_argument("--workload", default="starvla", choices=("starvla", "pi05", "pi05_fp8", "pi05_int8", "pi05_int4", "tiny"))
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--euler-steps", type=int, default=None, help="Euler steps per loop (default: workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -81,9 +81,12 @@ def algorithmic_bytes(d):
     """Bytes one loop must move from HBM: N x (linear weights (+ fp8 scales) + B x prefix K/V)."""
     H, I, qd, kd = d.hidden, d.inter, d.qd, d.kd
     params = H * (qd + 2 * kd) + H * qd + 2 * I * H + H * I
-    wb = params * (1 if d.wtype != "bf16" else 2)
-    if d.wtype != "bf16":
-        wb += 4 * ((qd + 2 * kd) + H + 2 * I + H)
+    if d.wtype == "int4_g128":   # half a byte per weight + one fp32 scale per row and 128 inputs
+        wb = params // 2 + 4 * ((qd + 2 * kd) * -(-H // 128) + H * -(-qd // 128) + 2 * I * -(-H // 128) + H * -(-I // 128))
+    else:
+        wb = params * (1 if d.wtype != "bf16" else 2)
+        if d.wtype != "bf16":
+            wb += 4 * ((qd + 2 * kd) + H + 2 * I + H)
     kv = 2 * d.n_prefix * kd * 2
     return d.steps * d.n_layers * (wb + d.batch * kv)
 
@@ -353,7 +356,8 @@ def run_native(args):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {"bf16": "bf16", "fp8_e4m3": "e4m3 weights x bf16 activations",
-                  "int8": "int8 weights x bf16 activations"}[d.wtype],
+                  "int8": "int8 weights x bf16 activations",
+                  "int4_g128": "int4 weights (groups of 128) x bf16 activations"}[d.wtype],
         "data": "synthetic", "config": {**workload_config(d, args), "engine": engine},
         "ms_per_loop": round(ms, 5),
         "actions_per_s": round(world * d.batch * d.n_action_tokens * 1000.0 / ms, 1),

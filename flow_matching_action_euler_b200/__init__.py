@@ -17,11 +17,11 @@ __all__ = [
     "lib", "VlaAeDims", "VlaAeWeights", "VlaAeTrace", "VlaAeError", "ActionExpert",
     "vla_ae_create", "vla_ae_set_prefix", "vla_ae_denoise", "vla_ae_denoise_host", "vla_ae_status",
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
-    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "vla_ae_denoise_sched", "vla_ae_set_prefix_next", "vla_ae_denoise_stale", "BF16", "FP8_E4M3", "INT8", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
+    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "vla_ae_denoise_sched", "vla_ae_set_prefix_next", "vla_ae_denoise_stale", "BF16", "FP8_E4M3", "INT8", "INT4_G128", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
     "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES", "Q_ENGINE", "ENGINE_PER_OP", "ENGINE_PERSISTENT",
 ]
 
-BF16, FP8_E4M3, INT8 = 0, 1, 2
+BF16, FP8_E4M3, INT8, INT4_G128 = 0, 1, 2, 3
 Q_KERNELS_PER_LOOP, Q_WEIGHT_BYTES, Q_KV_BYTES, Q_DEVICE_BYTES, Q_SPLITS, Q_OP_BYTES, Q_ENGINE = 1, 2, 3, 4, 5, 6, 7
 ENGINE_PER_OP, ENGINE_PERSISTENT = 0, 1
 OK, EINVAL, ENOMEM, ECUDA, ENOPREFIX, ETIMEOUT, EUNSUPPORTED = 0, -1, -2, -3, -4, -5, -6

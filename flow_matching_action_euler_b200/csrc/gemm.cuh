@@ -39,13 +39,14 @@ enum EpiKind : int { EPI_QKV = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
 constexpr int kGemmThreads = 192;
 constexpr int kMathThreads = 128;
 constexpr int kTileBytes = 16384;      // one packed weight tile
-constexpr int kConvStages = 2;         // fp8 path: converted bf16 A stages (2 x 16 KB each)
+constexpr int kConvStages = 2;         // packed-code paths: converted bf16 A stages (KPT x 16 KB each)
 constexpr int kMaxMpc = 4;             // m-tiles per CTA
 
 struct GemmParams {
   // ---- A operand (packed weights)
   const uint8_t* w;        // tiles [Mt][KBt][16 KB]
-  const float* wscale;     // fp8: scale per packed row (else nullptr)
+  const float* wscale;     // 8-bit codes: scale per packed row; int4: [packed row][spr] (else nullptr)
+  int spr;                 // scales per packed row (int4: one per 128 inputs)
   int Mt;                  // 128-row output tiles
   int mpc;                 // m-tiles per CTA (sharing the activation operand)
   int KBt;                 // weight tiles along K (64 wide for bf16, 128 wide for fp8)
@@ -109,7 +110,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
   const int mt0 = mg * mpc;
   const int nmt = min(mpc, p.Mt - mt0);
   const int kt0 = (r * p.KBt) / S, kt1 = ((r + 1) * p.KBt) / S, nkt = kt1 - kt0;
-  constexpr int KPT = FP8 ? 2 : 1;   // 64-wide k-blocks per weight tile
+  constexpr int KPT = WQ == 3 ? 4 : FP8 ? 2 : 1;   // 64-wide k-blocks per weight tile
+  constexpr bool ROW_SCALE = WQ == 1 || WQ == 2;     // scale applied in the epilogue
   const int kb0 = kt0 * KPT;
   const int kb1 = min(kt1 * KPT, p.KB);
   const int NT = p.NT;
@@ -245,12 +247,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
+          for (int half = 0; half < KPT; ++half) {
             const int lkb = li * 2 + half;                      // local 64-wide k-block
             if (kb0 + lkb >= kb1) break;                        // ragged K tail
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_k(d_tmem, sw128_desc(aBase + (c * 2 + half) * kTileBytes + kk * 32),
+              mma_k(d_tmem, sw128_desc(aBase + (c * KPT + half) * kTileBytes + kk * 32),
                     bBase + (uint32_t)lkb * 2u * bstride + kk * 32, (lkb | kk) != 0);
           }
           mma_commit(&cempty[c]);
@@ -264,13 +266,48 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
     const int mtid = threadIdx.x - 64;   // 0..127
     int conv_done = 0;
     auto convert_one = [&](int i) -> bool {
-      // 8-bit tile (128 rows x 128 B, swizzled by 16 B chunks) -> two bf16 SW128 tiles
+      // 8-bit tile (128 rows x 128 B, swizzled by 16 B chunks) -> two bf16 SW128 tiles;
+      // int4 tile (128 rows x 256 codes) -> four, each code times its group's scale
       const int s = i % p.stages, c = i % kConvStages;
+      float gsc[8];
+      if constexpr (WQ == 3) {   // the group scales of this thread's 8 chunks, before any wait
+        const int j = i / nkt, kt = kt0 + i % nkt;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int idx = mtid + jj * kMathThreads, row = idx >> 3, ch = idx & 7;
+          // chunks past K hold zero codes; their group index is clamped to stay inside the row
+          const int g = min(kt * 2 + (ch >> 2), p.spr - 1);
+          gsc[jj] = __ldg(p.wscale + (size_t)((mt0 + j) * 128 + row) * p.spr + g);
+        }
+      }
       if (!mbar_wait(&full[s], (i / p.stages) & 1, p.status, DEV_ERR_TIMEOUT_TMA)) return false;
       if (i >= kConvStages && !mbar_wait(&cempty[c], ((i / kConvStages) - 1) & 1, p.status, DEV_ERR_TIMEOUT_CONV))
         return false;
       const uint8_t* src = sA + (size_t)s * kTileBytes;
-      uint8_t* dst = sC + (size_t)c * 2 * kTileBytes;
+      uint8_t* dst = sC + (size_t)c * KPT * kTileBytes;
+      if constexpr (WQ == 3) {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int idx = mtid + jj * kMathThreads;   // 0..1023: (row, 32-code chunk)
+          const int row = idx >> 3, ch = idx & 7;
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + sw128_chunk_byte(row, ch));
+          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+          const float sc = gsc[jj];
+          uint8_t* t = dst + (ch >> 1) * kTileBytes;   // which 64-wide bf16 tile
+          const int bch = (ch & 1) * 4;                 // its first 8-element chunk
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {                 // codes 8q .. 8q+7 -> one bf16 chunk
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c0 = (int)((w4[q] >> (8 * e)) & 0xFu), c1 = (int)((w4[q] >> (8 * e + 4)) & 0xFu);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn((float)((c0 ^ 8) - 8) * sc, (float)((c1 ^ 8) - 8) * sc);
+              o[e] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(t + sw128_chunk_byte(row, bch + q)) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      } else {
 #pragma unroll 4
       for (int jj = 0; jj < 8; ++jj) {
         const int idx = mtid + jj * kMathThreads;   // 0..1023: (row, fp8 chunk)
@@ -289,6 +326,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
         *reinterpret_cast<uint4*>(t + sw128_chunk_byte(row, bch)) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4*>(t + sw128_chunk_byte(row, bch + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
       }
+      }
       fence_proxy_async_smem();
       mbar_arrive(&cfull[c]);
       mbar_arrive(&empty[s]);
@@ -303,7 +341,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
         v_gate[i] = in ? __ldg(p.gate + o) : 0.f;
         v_scn[i] = (in && p.sc_next) ? __ldg(p.sc_next + o) : 0.f;
       }
-      if (FP8) v_wsc[i] = in ? __ldg(p.wscale + o) : 0.f;
+      if (ROW_SCALE) v_wsc[i] = in ? __ldg(p.wscale + o) : 0.f;
     }
     bool ok = true;
     if (FP8) {
@@ -451,7 +489,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
         for (int q = 0; q < 16; ++q) y[q] += rr[(size_t)q * RST];
       }
       const int lr = o0 - mt0 * 128;            // row inside this CTA's staged vectors
-      if (FP8) {
+      if (ROW_SCALE) {
 #pragma unroll
         for (int q = 0; q < 16; ++q) y[q] *= v_wsc[lr + q];
       }

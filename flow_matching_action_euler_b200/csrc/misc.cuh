@@ -259,6 +259,42 @@ __global__ void quant_int8_kernel(const __nv_bfloat16* const* __restrict__ rows,
   }
 }
 
+// Group-wise symmetric int4 packing (W4A16): per row and group of 128 inputs, scale = max|w| / 7
+// (1 for a zero group), code = round-to-nearest-even(w / scale) clamped to [-7, 7].  Tiles hold
+// 128 rows x 256 codes (two per byte, low nibble first), 16-byte chunks of 32 codes swizzled;
+// scales [row][ceil(K / 128)].  One warp per row.
+__global__ void quant_int4_kernel(const __nv_bfloat16* const* __restrict__ rows, int K, int Mt, int KB4,
+                                  uint8_t* __restrict__ dst, float* __restrict__ scales) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= Mt * 128) return;
+  const __nv_bfloat16* src = rows[row];
+  const int ng = (K + 127) / 128;
+  for (int g = lane; g < ng; g += 32) {
+    float amax = 0.f;
+    if (src)
+      for (int k = g * 128; k < min(K, g * 128 + 128); ++k) amax = fmaxf(amax, fabsf(__bfloat162float(src[k])));
+    scales[(size_t)row * ng + g] = amax == 0.f ? 1.f : __fdiv_rn(amax, 7.f);
+  }
+  __syncwarp();
+  const int mt = row >> 7, r = row & 127;
+  for (int c = lane; c < KB4 * 8; c += 32) {            // 32-code chunks along K
+    const int kb = c >> 3, ch = c & 7, k0 = c * 32;
+    uint32_t word[4] = {0, 0, 0, 0};
+    if (src && k0 < K) {   // (chunks past K keep zero codes)
+      const float sc = scales[(size_t)row * ng + k0 / 128];   // written by this warp above
+#pragma unroll 8
+      for (int q = 0; q < 32; ++q) {
+        const int k = k0 + q;
+        const float v = k < K ? rintf(__fdiv_rn(__bfloat162float(src[k]), sc)) : 0.f;   // ties to even
+        const int code = max(-7, min(7, (int)v));
+        word[q >> 3] |= (uint32_t)(code & 0xF) << ((q & 7) * 4);
+      }
+    }
+    *reinterpret_cast<uint4*>(dst + ((size_t)mt * KB4 + kb) * kTileBytesPack + sw128_chunk_byte(r, ch)) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+  }
+}
+
 // ---------------------------------------------------------------- prefix layout (set_prefix)
 // user K, V: [B][L][P][nkv][hd]  ->  K cache [L][B][nkv][Lpad][hd], V^T cache [L][B][nkv][hd][Lpad]
 __global__ void prefix_layout_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
@@ -328,7 +364,7 @@ __global__ void untile_kernel(const __nv_bfloat16* tiles, float* out, int Ntok, 
 // out[k][pr] = sum_c W[pr][c] shift_k[c], with W read back from the packed tiles (8-bit formats:
 // decoded code times the row scale, i.e. exactly the weights the GEMM multiplies).  One warp per row.
 __global__ void cshift_kernel(const uint8_t* __restrict__ wt, const float* __restrict__ wscale, int rows, int KBt,
-                              int K, int wq, const float* __restrict__ shift, size_t shift_step_stride, int steps,
+                              int K, int wq, int spr, const float* __restrict__ shift, size_t shift_step_stride, int steps,
                               float* out, size_t out_step_stride) {
   const int pr = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (pr >= rows) return;
@@ -338,7 +374,12 @@ __global__ void cshift_kernel(const uint8_t* __restrict__ wt, const float* __res
     const float* sh = shift + (size_t)k * shift_step_stride;
     for (int c = lane; c < K; c += 32) {
       float w;
-      if (wq) {   // 8-bit codes (1: e4m3, 2: int8) times the row scale
+      if (wq == 3) {   // int4 code times its group's scale, rounded to bf16 as the GEMM widens it
+        const uint8_t* tile = wt + ((size_t)mt * KBt + c / 256) * kTileBytesPack;
+        const int kk = c % 256;
+        const int nib = (tile[sw128_chunk_byte(r, kk / 32) + (kk % 32) / 2] >> (4 * (kk & 1))) & 0xF;
+        w = __bfloat162float(__float2bfloat16_rn((float)((nib ^ 8) - 8) * wscale[(size_t)pr * spr + c / 128]));
+      } else if (wq) {   // 8-bit codes (1: e4m3, 2: int8) times the row scale
         const uint8_t* tile = wt + ((size_t)mt * KBt + c / 128) * kTileBytesPack;
         const uint8_t code = tile[sw128_chunk_byte(r, (c % 128) / 16) + (c % 16)];
         const uint32_t pair = wq == 2 ? s8x2_to_bf16x2((uint16_t)code) : e4m3x2_to_bf16x2((uint16_t)code);

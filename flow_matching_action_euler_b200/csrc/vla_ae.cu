@@ -191,10 +191,15 @@ cudaError_t launch_coop(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStr
 
 using GemmKernel = void (*)(const GemmParams);
 
+// 64-wide k-blocks per packed weight tile of weight format wq (0 bf16, 1 e4m3, 2 int8, 3 int4)
+int wq_kpt(int wq) { return wq == 3 ? 4 : wq ? 2 : 1; }
+// fp32 scales per packed row of an op with K inputs: 1 (e4m3, int8), one per 128 inputs (int4)
+int wq_scales_per_row(int wq, int K) { return wq == 3 ? ceil_div(K, 128) : 1; }
+
 template <int EPI, bool NORM>
 GemmKernel gemm_kernel_wq(int wq) {
-  return wq == 2 ? gemm_stream_kernel<EPI, 2, NORM> : wq == 1 ? gemm_stream_kernel<EPI, 1, NORM>
-                                                                : gemm_stream_kernel<EPI, 0, NORM>;
+  return wq == 3 ? gemm_stream_kernel<EPI, 3, NORM> : wq == 2 ? gemm_stream_kernel<EPI, 2, NORM>
+         : wq == 1 ? gemm_stream_kernel<EPI, 1, NORM> : gemm_stream_kernel<EPI, 0, NORM>;
 }
 GemmKernel gemm_kernel_for(OpId id, int wq) {
   switch (id) {
@@ -222,16 +227,18 @@ AttnKernel attn_kernel_for(int hd, int cs) {
 }
 
 // shared-memory layout of one GEMM op for a given (m-tiles per CTA, split, ring depth)
-void gemm_layout(OpPlan& p, int NT, bool fp8) {
+// kpt: 64-wide k-blocks per packed weight tile (1 bf16, 2 e4m3 / int8, 4 int4)
+void gemm_layout(OpPlan& p, int NT, int kpt) {
+  const bool fp8 = kpt > 1;
   const int nkt_max = ceil_div(p.KBt, p.S);
-  const int nkb_max = std::min(nkt_max * (fp8 ? 2 : 1), p.KB);
+  const int nkb_max = std::min(nkt_max * kpt, p.KB);
   const size_t b_region = (size_t)2 * nkb_max * NT * 128;
   // split-K receive buffer [S][16 ceil(8 mpc / S)][NT + 4] fp32, over ring + operand
   const size_t red = (size_t)p.S * 16 * ceil_div(8 * p.mpc, p.S) * (NT + 4) * 4;
   size_t a_region = (size_t)p.stages * kTileBytes;
   if (a_region + b_region < red) a_region = red - b_region;
   a_region = align_up(a_region, 1024);
-  const size_t conv = fp8 ? (size_t)kConvStages * 2 * kTileBytes : 0;
+  const size_t conv = fp8 ? (size_t)kConvStages * kpt * kTileBytes : 0;
   p.off_b = (int)a_region;
   p.off_conv = (int)(a_region + align_up(b_region, 1024));
   p.off_bar = (int)(p.off_conv + conv);
@@ -274,7 +281,8 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
   base.K = K;
   base.Mt = ceil_div(O, 128);
   base.KB = ceil_div(K, 64);
-  base.KBt = fp8 ? ceil_div(K, 128) : base.KB;
+  const int kpt = wq_kpt(H->wq);
+  base.KBt = ceil_div(K, 64 * kpt);
   base.wbytes = (size_t)base.Mt * base.KBt * kTileBytes;
   GemmKernel kern = gemm_kernel_for(id, H->wq);
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
@@ -300,11 +308,11 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
         const int tiles = mpc * ceil_div(base.KBt, S);
         // deepest ring inside the budget (at least 2 stages when there is more than one tile)
         p.stages = 1;
-        gemm_layout(p, H->NT, fp8);
+        gemm_layout(p, H->NT, kpt);
         for (int st = 2; st <= std::min(tiles, 8); ++st) {
           OpPlan t = p;
           t.stages = st;
-          gemm_layout(t, H->NT, fp8);
+          gemm_layout(t, H->NT, kpt);
           if (t.smem > (fp8 ? kMaxDynSmem : budget) && p.stages >= 2) break;
           if (t.smem > kMaxDynSmem) break;
           p = t;
@@ -371,7 +379,9 @@ int validate_dims(const vla_ae_dims* d) {
   if (d->action_dim > kMaxAction) return VLA_AE_EINVAL;
   if ((long long)d->batch * (d->n_action_tokens + d->has_state_token) > 4096) return VLA_AE_EINVAL;
   if (!(d->rope_theta > 0.f) || !(d->rms_eps >= 0.f)) return VLA_AE_EINVAL;
-  if (d->wtype != VLA_AE_BF16 && d->wtype != VLA_AE_FP8_E4M3 && d->wtype != VLA_AE_INT8) return VLA_AE_EINVAL;
+  if (d->wtype != VLA_AE_BF16 && d->wtype != VLA_AE_FP8_E4M3 && d->wtype != VLA_AE_INT8 &&
+      d->wtype != VLA_AE_INT4_G128)
+    return VLA_AE_EINVAL;
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return VLA_AE_EUNSUPPORTED;
   return VLA_AE_OK;
 }
@@ -636,6 +646,7 @@ GemmParams gemm_common(const vla_ae* H, OpId id, int layer) {
   set_prefetch(H, g, id, layer);
   g.w = H->wpack + (size_t)layer * H->layer_wbytes + p.woff;
   g.wscale = H->fp8 ? H->wscale + (size_t)layer * H->layer_scales + p.soff : nullptr;
+  g.spr = wq_scales_per_row(H->wq, p.K);
   g.Mt = p.Mt;
   g.mpc = p.mpc;
   g.KBt = p.KBt;
@@ -948,11 +959,11 @@ int get_tables_grid(vla_ae* H, const std::vector<double>& grid, bool uniform, St
     const size_t mstep = (size_t)d.n_layers * 6 * Hd;
     const OpPlan& pq = H->op[OP_QKV];
     cshift_kernel<<<ceil_div((int)rq, 8), 256, 0, H->cap>>>(wl + pq.woff, sl ? sl + pq.soff : nullptr, (int)rq, pq.KBt,
-                                                           pq.K, H->wq, mod_l + 0 * Hd, mstep, steps,
+                                                           pq.K, H->wq, wq_scales_per_row(H->wq, pq.K), mod_l + 0 * Hd, mstep, steps,
                                                            T.cq + (size_t)l * rq, (size_t)d.n_layers * rq);
     const OpPlan& pg = H->op[OP_GU];
     cshift_kernel<<<ceil_div((int)rg, 8), 256, 0, H->cap>>>(wl + pg.woff, sl ? sl + pg.soff : nullptr, (int)rg, pg.KBt,
-                                                           pg.K, H->wq, mod_l + 3 * Hd, mstep, steps,
+                                                           pg.K, H->wq, wq_scales_per_row(H->wq, pg.K), mod_l + 3 * Hd, mstep, steps,
                                                            T.cg + (size_t)l * rg, (size_t)d.n_layers * rg);
   }
   CK(cudaGetLastError());
@@ -1068,7 +1079,10 @@ int pack_weights(vla_ae* H, const vla_ae_weights* w) {
       }
       CK(cudaMemcpy(rowptr_dev, rows.data(), (size_t)p.Mt * 128 * sizeof(void*), cudaMemcpyHostToDevice));
       uint8_t* dst = H->wpack + (size_t)l * H->layer_wbytes + p.woff;
-      if (H->wq == 2) {
+      if (H->wq == 3) {
+        quant_int4_kernel<<<ceil_div(p.Mt * 128, 8), 256>>>(rowptr_dev, p.K, p.Mt, p.KBt, dst,
+                                                           H->wscale + (size_t)l * H->layer_scales + p.soff);
+      } else if (H->wq == 2) {
         quant_int8_kernel<<<ceil_div(p.Mt * 128, 8), 256>>>(rowptr_dev, p.K, p.Mt, p.KBt, dst,
                                                            H->wscale + (size_t)l * H->layer_scales + p.soff);
       } else if (H->wq == 1) {
@@ -1090,7 +1104,7 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
   int rc;
   H->d = *dims;
   const vla_ae_dims& d = H->d;
-  H->wq = d.wtype == VLA_AE_FP8_E4M3 ? 1 : d.wtype == VLA_AE_INT8 ? 2 : 0;
+  H->wq = d.wtype == VLA_AE_FP8_E4M3 ? 1 : d.wtype == VLA_AE_INT8 ? 2 : d.wtype == VLA_AE_INT4_G128 ? 3 : 0;
   H->fp8 = H->wq != 0;
   CK(cudaGetDevice(&H->device));
   CK(cudaDeviceGetAttribute(&H->num_sms, cudaDevAttrMultiProcessorCount, H->device));
@@ -1117,7 +1131,7 @@ int create_impl(const vla_ae_dims* dims, const vla_ae_weights* w, vla_ae* H) {
     H->op[id].woff = woff;
     H->op[id].soff = soff;
     woff += H->op[id].wbytes;
-    soff += (size_t)H->op[id].Mt * 128;
+    soff += (size_t)H->op[id].Mt * 128 * wq_scales_per_row(H->wq, H->op[id].K);
   }
   H->layer_wbytes = woff;
   H->layer_scales = soff;
@@ -1399,8 +1413,9 @@ int vla_ae_query(vla_ae_t H, int what, int arg, long long* value) {
         return VLA_AE_OK;
       }
       const OpId id = arg == 0 ? OP_QKV : arg == 2 ? OP_O : arg == 3 ? OP_GU : OP_D;
-      long long b = (long long)H->op[id].O * H->op[id].K * (H->fp8 ? 1 : 2);
-      if (H->fp8) b += 4LL * H->op[id].O;
+      const long long ok = (long long)H->op[id].O * H->op[id].K;
+      long long b = H->wq == 3 ? (ok + 1) / 2 : ok * (H->fp8 ? 1 : 2);
+      if (H->fp8) b += 4LL * H->op[id].O * wq_scales_per_row(H->wq, H->op[id].K);
       *value = b;
       return VLA_AE_OK;
     }
@@ -1524,8 +1539,9 @@ int vla_ae_debug_weight(vla_ae_t H, int layer, int which, void* w_host, float* s
   std::vector<uint8_t> blob(p.wbytes);
   CK(cudaMemcpy(blob.data(), H->wpack + (size_t)layer * H->layer_wbytes + p.woff, p.wbytes, cudaMemcpyDeviceToHost));
   std::vector<float> sc;
+  const int spr = wq_scales_per_row(H->wq, p.K);
   if (H->fp8) {
-    sc.resize((size_t)p.Mt * 128);
+    sc.resize((size_t)p.Mt * 128 * spr);
     CK(cudaMemcpy(sc.data(), H->wscale + (size_t)layer * H->layer_scales + p.soff, sc.size() * 4,
                   cudaMemcpyDeviceToHost));
   }
@@ -1536,7 +1552,13 @@ int vla_ae_debug_weight(vla_ae_t H, int layer, int which, void* w_host, float* s
     if (mat != which) continue;
     const int mt = pr / 128, r = pr % 128;
     for (int k = 0; k < K; ++k) {
-      if (H->fp8) {
+      if (H->wq == 3) {   // int4: two codes per byte (low nibble first), returned one per byte
+        const size_t tile = (size_t)mt * p.KBt + k / 256;
+        const int kk = k % 256;
+        const size_t byte = tile * kTileBytes + sw128_chunk_byte(r, kk / 32) + (kk % 32) / 2;
+        const int nib = (blob[byte] >> (4 * (kk & 1))) & 0xF;
+        reinterpret_cast<int8_t*>(w_host)[(size_t)row * K + k] = (int8_t)((nib ^ 8) - 8);
+      } else if (H->fp8) {
         const size_t tile = (size_t)mt * p.KBt + k / 128;
         const int kk = k % 128;
         const size_t byte = tile * kTileBytes + sw128_chunk_byte(r, kk / 16) + (kk % 16);
@@ -1547,7 +1569,8 @@ int vla_ae_debug_weight(vla_ae_t H, int layer, int which, void* w_host, float* s
         reinterpret_cast<uint16_t*>(w_host)[(size_t)row * K + k] = reinterpret_cast<const uint16_t*>(blob.data())[elem];
       }
     }
-    if (H->fp8 && scales_host) scales_host[row] = sc[pr];
+    if (H->fp8 && scales_host)
+      for (int g = 0; g < spr; ++g) scales_host[(size_t)row * spr + g] = sc[(size_t)pr * spr + g];
   }
   return VLA_AE_OK;
 }

@@ -42,8 +42,10 @@ extern "C" {
 /* ------------------------------------------------------------------ configuration */
 /* Weight formats of the per-layer linears.  FP8_E4M3: the FP8 weights of the APXInf article
  * (section "CUDA Graph、FP8 和 Rust").  INT8: the INT8 quantisation the same section names for
- * GPUs without FP8 tensor cores (Jetson Orin), here weight-only with one scale per output channel. */
-typedef enum { VLA_AE_BF16 = 0, VLA_AE_FP8_E4M3 = 1, VLA_AE_INT8 = 2 } vla_ae_wtype;
+ * GPUs without FP8 tensor cores (Jetson Orin), here weight-only with one scale per output channel.
+ * INT4_G128: INT4, named next to FP8 in "AI Infra如何优化VLA" (section 后续工作), here W4A16 with
+ * one scale per output channel and group of 128 inputs. */
+typedef enum { VLA_AE_BF16 = 0, VLA_AE_FP8_E4M3 = 1, VLA_AE_INT8 = 2, VLA_AE_INT4_G128 = 3 } vla_ae_wtype;
 
 /* Model and workload dimensions, fixed at create time.
  * Requirements (else VLA_AE_EINVAL): every count >= 1 except has_state_token (0/1) and
@@ -78,8 +80,10 @@ typedef struct {
  * library quantises q/k/v/o/gate/up/down itself (one fp32 scale per output channel, scale =
  * max|w|/448, codes = e4m3 round-to-nearest-even saturating of w/scale); with wtype INT8 likewise
  * with scale = max|w|/127 and codes = round-to-nearest-even of w/scale clamped to [-127, 127]
- * (a zero row takes scale 1); everything else stays bf16.  The caller keeps ownership; the
- * library copies. */
+ * (a zero row takes scale 1); with wtype INT4_G128 per output channel and group of 128 inputs
+ * with scale = max|w_group|/7 and codes clamped to [-7, 7], the tensor cores then multiply
+ * bf16(code * scale); everything else stays bf16.  The caller keeps ownership; the library
+ * copies. */
 typedef struct {
   const void *w_in, *b_in, *w_state, *b_state;
   const void *const *w_ada, *const *b_ada;
@@ -243,9 +247,9 @@ int vla_ae_debug_wait_probe(vla_ae_t h, unsigned attempts);
 int vla_ae_debug_velocity(vla_ae_t h, int step, int steps, const float *x, float *v);
 
 /* Read back one packed per-layer weight in [out][in] order (which: 0 q, 1 k, 2 v, 3 o, 4 gate,
- * 5 up, 6 down) into host memory: bf16 weights as uint16 bits, FP8 / INT8 weights as their
- * 8-bit codes (e4m3 bits / two's-complement int8) plus fp32 scales [out] (scales may be NULL for
- * bf16).  Synchronous. */
+ * 5 up, 6 down) into host memory: bf16 weights as uint16 bits, FP8 / INT8 / INT4 weights as
+ * one code per byte (e4m3 bits / two's-complement int8 / int4 sign-extended to int8) plus fp32
+ * scales [out] ([out][ceil(in/128)] for INT4; scales may be NULL for bf16).  Synchronous. */
 int vla_ae_debug_weight(vla_ae_t h, int layer, int which, void *w_host, float *scales_host);
 
 #ifdef __cplusplus

@@ -30,6 +30,9 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
                        matrix, P = 0, constant-V rows, MHA case
 ``linear``/``swiglu``  torch float64 linear / silu, SiLU(0) = 0
 ``e4m3_*``             exhaustive code table, RNE ties, saturation, torch cast
+``*_int4``             per 128-input group: the max entry maps to +-7, ties to
+                       even, zero groups, ragged last group, torch's round on
+                       the quotients and torch's bf16 cast of code * scale
 ``*_int8``             the max entry maps to +-127, integer multiples of the
                        scale round-trip, half-to-even ties, zero rows, torch's
                        round on the same quotients, |W' - W| <= scale / 2
@@ -50,3 +53,4 @@ from .fp8 import (  # noqa: F401
     e4m3_decode, e4m3_encode, quantize_rowwise_e4m3, dequantize_rowwise_e4m3,
 )
 from .int8 import quantize_rowwise_int8, dequantize_rowwise_int8  # noqa: F401
+from .int4 import quantize_groupwise_int4, dequantize_groupwise_int4  # noqa: F401

@@ -28,6 +28,7 @@ import numpy as np
 
 from .fp8 import quantize_rowwise_e4m3, dequantize_rowwise_e4m3
 from .int8 import quantize_rowwise_int8, dequantize_rowwise_int8
+from .int4 import quantize_groupwise_int4, dequantize_groupwise_int4
 
 
 def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
@@ -189,8 +190,9 @@ class OracleWeights:
     """float64 view of the synthetic bf16 weights (optionally with dequantised 8-bit linears).
 
     ``quantized`` = ``"fp8_e4m3"`` (or ``True``) replaces each per-layer q/k/v/o/gate/up/down
-    weight W by W' = e4m3(W / s) * s, ``"int8"`` by W' = round(W / s) * s, with one scale per
-    output channel; adaLN, in/out/state projections stay bf16.  ``False`` / ``"bf16"``: none.
+    weight W by W' = e4m3(W / s) * s, ``"int8"`` by W' = round(W / s) * s (one scale per output
+    channel), ``"int4_g128"`` by W' = bf16(round(W / s) * s) (one scale per output channel and
+    128 inputs); adaLN, in/out/state projections stay bf16.  ``False`` / ``"bf16"``: none.
     """
 
     def __init__(self, w: Dict[str, object], d, quantized=False):
@@ -198,7 +200,7 @@ class OracleWeights:
         if quantized is True:
             quantized = "fp8_e4m3"
         self.quantized = False if quantized in (False, None, "bf16") else quantized
-        if self.quantized not in (False, "fp8_e4m3", "int8"):
+        if self.quantized not in (False, "fp8_e4m3", "int8", "int4_g128"):
             raise ValueError(f"unknown weight format {quantized!r}")
         self._raw = w
         self.top = {k: bf16_to_f64(v) for k, v in w.items() if k != "layers"}
@@ -217,6 +219,10 @@ class OracleWeights:
             for k in _LAYER_LINEARS:
                 codes, scales = quantize_rowwise_int8(lw[k].astype(np.float32))
                 lw[k] = dequantize_rowwise_int8(codes, scales)
+        elif self.quantized == "int4_g128":
+            for k in _LAYER_LINEARS:
+                codes, scales = quantize_groupwise_int4(lw[k].astype(np.float32))
+                lw[k] = dequantize_groupwise_int4(codes, scales)
         self._cache[l] = lw
         return lw
 

@@ -19,6 +19,8 @@ Workload shapes follow the five workloads the action expert is measured on:
                   fp32 scales), 1 or 10 steps.
 * ``pi05_int8`` -- ``pi05`` with int8 linear weights (per-output-channel
                   fp32 scales; the INT8 fallback of the same article).
+* ``pi05_int4`` -- ``pi05`` with int4 linear weights (W4A16, fp32 scales per
+                  output channel and 128 inputs).
 * batch sweep  -- ``tiny`` and ``starvla`` at batch 1, 4, 16 and 64.
 
 Random numbers: numpy's PCG64 bit generator (O'Neill, "PCG: A Family of
@@ -61,7 +63,7 @@ class Dims:
     n_prefix: int
     steps: int
     batch: int = 1
-    wtype: str = "bf16"          # "bf16", "fp8_e4m3" or "int8"
+    wtype: str = "bf16"          # "bf16", "fp8_e4m3", "int8" or "int4_g128"
     rope_theta: float = 10000.0
     rms_eps: float = 1e-6
 
@@ -98,6 +100,9 @@ CONFIGS: Dict[str, Dims] = {
     "pi05_int8": Dims(n_layers=18, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=256,
                       inter=4096, t_emb_dim=256, action_dim=32, n_action_tokens=50,
                       has_state_token=0, n_prefix=800, steps=10, wtype="int8"),
+    "pi05_int4": Dims(n_layers=18, hidden=1024, n_q_heads=8, n_kv_heads=1, head_dim=256,
+                      inter=4096, t_emb_dim=256, action_dim=32, n_action_tokens=50,
+                      has_state_token=0, n_prefix=800, steps=10, wtype="int4_g128"),
 }
 
 BATCH_SWEEP = (1, 4, 16, 64)
@@ -225,4 +230,4 @@ def abi_dims(d: Dims, max_prefix: int | None = None) -> Dict[str, object]:
                 head_dim=d.head_dim, inter=d.inter, t_emb_dim=d.t_emb_dim, action_dim=d.action_dim,
                 n_action_tokens=d.n_action_tokens, has_state_token=d.has_state_token,
                 max_prefix=d.n_prefix if max_prefix is None else max_prefix, batch=d.batch,
-                rope_theta=d.rope_theta, rms_eps=d.rms_eps, wtype={"bf16": 0, "fp8_e4m3": 1, "int8": 2}[d.wtype])
+                rope_theta=d.rope_theta, rms_eps=d.rms_eps, wtype={"bf16": 0, "fp8_e4m3": 1, "int8": 2, "int4_g128": 3}[d.wtype])

@@ -70,7 +70,8 @@ def test_full_size_bf16(name):
         c.close()
 
 
-@pytest.mark.parametrize("wtype,steps", [("pi05_fp8", 1), ("pi05_fp8", 10), ("pi05_int8", 1), ("pi05_int8", 10)])
+@pytest.mark.parametrize("wtype,steps", [("pi05_fp8", 1), ("pi05_fp8", 10), ("pi05_int8", 1), ("pi05_int8", 10),
+                                         ("pi05_int4", 1), ("pi05_int4", 10)])
 def test_full_size_fp8(wtype, steps):
     c = Case(config(wtype, steps=steps))
     try:
@@ -78,7 +79,8 @@ def test_full_size_fp8(wtype, steps):
         ref_q = c.oracle_denoise()
         assert rel_err(got, ref_q) <= 2e-2
         ref_bf16 = c.oracle_denoise(W=oracle.OracleWeights(c.w, c.d, quantized=False))
-        assert rel_err(got, ref_bf16) <= 5e-2
+        # 8-bit formats within 5e-2 of the bf16-weight oracle; int4 (W4A16) is looser
+        assert rel_err(got, ref_bf16) <= (0.25 if c.d.wtype == "int4_g128" else 5e-2)
     finally:
         c.close()
 

@@ -350,6 +350,30 @@ def test_fp8_tiny():
     assert rel_err(got, ref_bf16) <= FP8_TOL
 
 
+def test_int4_codes_and_scales_bitexact():
+    c = case("ragged", wtype="int4_g128")
+    for layer in range(c.d.n_layers):
+        for which, key in enumerate(("wq", "wk", "wv", "wo", "wg", "wu", "wd")):
+            w32 = oracle.bf16_to_f64(c.w["layers"][layer][key]).astype(np.float32)
+            codes, scales = oracle.quantize_groupwise_int4(w32)
+            got = np.zeros(codes.shape, np.int8)
+            gs = np.zeros(scales.shape, np.float32)
+            c.ae.debug_weight(layer, which, got, gs)
+            assert np.array_equal(gs.view(np.uint32), scales.view(np.uint32)), (layer, key)
+            assert np.array_equal(got, codes), (layer, key, int(np.sum(got != codes)))
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_int4(name):
+    """W4A16: parity against the oracle on the same dequantised bf16 weights; the distance to the
+    bf16-weight oracle is the quantisation error (reported, loosely bounded)."""
+    c = case(name, wtype="int4_g128")
+    got = c.denoise()
+    assert rel_err(got, c.oracle_denoise()) <= 2e-2
+    assert rel_err(got, c.oracle_denoise(W=oracle.OracleWeights(c.w, c.d, quantized=False))) <= 0.25
+    _layer_check(c, 0, c.d.steps, layers=[0])
+
+
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
 def test_int8(name):
     c = case(name, wtype="int8")

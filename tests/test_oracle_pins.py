@@ -548,3 +548,36 @@ def test_int8_zero_row_and_torch_round():
     q = torch.from_numpy(w) / torch.from_numpy(scales)[:, None]
     want = torch.clamp(torch.round(q), -127, 127).to(torch.int8).numpy()
     np.testing.assert_array_equal(codes, want)
+
+
+# ----------------------------------------------------------------- INT4 weights (groups of 128)
+
+def test_int4_groups_max_maps_to_7_and_ragged_last_group():
+    w = RNG.standard_normal((16, 300)).astype(np.float32) * 0.02     # groups of 128, 128, 44
+    codes, scales = oracle.quantize_groupwise_int4(w)
+    assert codes.shape == (16, 300) and scales.shape == (16, 3)
+    assert codes.min() >= -7 and codes.max() <= 7
+    for g, (a, b) in enumerate(((0, 128), (128, 256), (256, 300))):
+        amax = np.max(np.abs(w[:, a:b]), axis=1)
+        np.testing.assert_array_equal(scales[:, g], (amax / np.float32(7.0)).astype(np.float32))
+        arg = a + np.argmax(np.abs(w[:, a:b]), axis=1)
+        np.testing.assert_array_equal(np.abs(codes[np.arange(16), arg]), 7)
+
+
+def test_int4_ties_zero_group_and_torch():
+    row = np.zeros((1, 256), np.float32)
+    row[0, :8] = [7.0, -7.0, 2.5, 3.5, -2.5, 0.5, 1.5, 6.5]     # group 0: scale exactly 1
+    codes, scales = oracle.quantize_groupwise_int4(row)
+    assert scales[0, 0] == 1.0 and scales[0, 1] == 1.0             # group 1 is all zero
+    np.testing.assert_array_equal(codes[0, :8], [7, -7, 2, 4, -2, 0, 2, 6])
+    assert not codes[0, 128:].any()
+    w = RNG.standard_normal((8, 256)).astype(np.float32)
+    codes, scales = oracle.quantize_groupwise_int4(w)
+    s = torch.from_numpy(scales).repeat_interleave(128, dim=1)
+    want = torch.clamp(torch.round(torch.from_numpy(w) / s), -7, 7).to(torch.int8).numpy()
+    np.testing.assert_array_equal(codes, want)
+    # the dequantised weight is torch's bf16 cast of the fp32 product
+    deq = oracle.dequantize_groupwise_int4(codes, scales)
+    want_deq = (torch.from_numpy(codes).float() * s).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(deq, want_deq)
+    assert np.all(np.abs(deq - w) <= s.numpy() * 0.5 * (1 + 2 ** -7) + 1e-30)
