@@ -36,6 +36,8 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
 ``*_int8``             the max entry maps to +-127, integer multiples of the
                        scale round-trip, half-to-even ties, zero rows, torch's
                        round on the same quotients, |W' - W| <= scale / 2
+``prefix_kv``          composed of the pinned rms_norm / linear / rope_half;
+                       invariant to scaling h; position 0 is the plain projection
 ``dit_layer``          zero gates give the identity, joint prefix permutation
                        invariance
 ``velocity``/``denoise``  parity unpinned beyond the parts above: batch
@@ -46,7 +48,7 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
 from .model import (  # noqa: F401
     bf16_to_f64, t_schedule, timestep_embedding, silu, rms_norm, modulate, rope_half,
     rope_positions_angles, gqa_attention, linear, swiglu, euler_integrate, euler_integrate_grid,
-    check_t_grid, uniform_grid, euler_integrate_switch, denoise_stale,
+    check_t_grid, uniform_grid, euler_integrate_switch, denoise_stale, prefix_kv,
     adaln_table, dit_layer, embed_tokens, velocity, denoise, denoise_batch, OracleWeights,
 )
 from .fp8 import (  # noqa: F401

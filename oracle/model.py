@@ -181,6 +181,19 @@ def swiglu(x: np.ndarray, wg: np.ndarray, wu: np.ndarray) -> np.ndarray:
     return silu(linear(x, wg)) * linear(x, wu)
 
 
+def prefix_kv(h: np.ndarray, wk: np.ndarray, wv: np.ndarray, gain: np.ndarray, n_kv_heads: int,
+              eps: float = 1e-6, theta: float = 10000.0):
+    """The VLM side of the cached prefix for one layer ("AI Infra如何优化VLA", section 算子开发: the
+    RMSNorm, K/V projection and RoPE of the prefill).  h [P, Hv] are the layer's input hidden
+    states of the P prefix tokens; x = rms_norm(h) * gain; K = rope_half(x Wk^T) at positions
+    0..P-1, V = x Wv^T; returns K, V as [P, n_kv_heads, hd]."""
+    x = rms_norm(h, eps) * gain
+    P = h.shape[0]
+    k = linear(x, wk).reshape(P, n_kv_heads, -1)
+    v = linear(x, wv).reshape(P, n_kv_heads, -1)
+    return rope_half(k, np.arange(P, dtype=np.float64), theta), v
+
+
 # ------------------------------------------------------------------ weights
 
 _LAYER_LINEARS = ("wq", "wk", "wv", "wo", "wg", "wu", "wd")

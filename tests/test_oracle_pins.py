@@ -581,3 +581,28 @@ def test_int4_ties_zero_group_and_torch():
     want_deq = (torch.from_numpy(codes).float() * s).to(torch.bfloat16).double().numpy()
     np.testing.assert_array_equal(deq, want_deq)
     assert np.all(np.abs(deq - w) <= s.numpy() * 0.5 * (1 + 2 ** -7) + 1e-30)
+
+
+# ----------------------------------------------------------------- prefix K/V producer
+
+def test_prefix_kv_invariants():
+    rng = np.random.default_rng(21)
+    P, Hv, nkv, hd = 9, 48, 2, 16
+    h = rng.standard_normal((P, Hv))
+    wk = rng.standard_normal((nkv * hd, Hv)) * 0.1
+    wv = rng.standard_normal((nkv * hd, Hv)) * 0.1
+    g = 1.0 + 0.1 * rng.standard_normal(Hv)
+    k, v = oracle.prefix_kv(h, wk, wv, g, nkv)
+    assert k.shape == (P, nkv, hd) and v.shape == (P, nkv, hd)
+    # RMSNorm makes the result invariant to a per-token scale of h (eps = 0)
+    k2, v2 = oracle.prefix_kv(h * np.linspace(0.5, 3.0, P)[:, None], wk, wv, g, nkv, eps=0.0)
+    k0, v0 = oracle.prefix_kv(h, wk, wv, g, nkv, eps=0.0)
+    np.testing.assert_allclose(k2, k0, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(v2, v0, rtol=1e-12, atol=1e-12)
+    # position 0 is not rotated; every position keeps the per-pair norms of the projection
+    x = h / np.sqrt(np.mean(h * h, axis=1, keepdims=True) + 1e-6) * g
+    kp = (x @ wk.T).reshape(P, nkv, hd)
+    np.testing.assert_allclose(k[0], kp[0], rtol=1e-12, atol=1e-12)
+    pair = lambda a: a[..., : hd // 2] ** 2 + a[..., hd // 2:] ** 2
+    np.testing.assert_allclose(pair(k), pair(kp), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(v, (x @ wv.T).reshape(P, nkv, hd), rtol=1e-12, atol=1e-12)
