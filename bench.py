@@ -390,6 +390,42 @@ def run_native(args):
                              "kernels_per_loop": int(ae.query(fm.Q_KERNELS_PER_LOOP, N))}
         ae.set_engine(fm.ENGINE_PERSISTENT if engine == "persistent" else fm.ENGINE_PER_OP)
         line["engines"] = engines
+        # prefix K/V producer (backbone RMSNorm + K/V projection + RoPE), synthetic backbone of
+        # width 2048: the compute-bound neighbour stage, against the tensor-core peak
+        if d.wtype == "bf16":
+            Hv = 2048
+            rng = np.random.default_rng(11)
+            from synth import f32_to_bf16_bits
+            mk = lambda shape, sd: f32_to_bf16_bits((rng.standard_normal(shape) * sd).astype(np.float32))
+            wk = [mk((d.kd, Hv), 0.02) for _ in range(d.n_layers)]
+            wv = [mk((d.kd, Hv), 0.02) for _ in range(d.n_layers)]
+            gn = [f32_to_bf16_bits((1.0 + 0.1 * rng.standard_normal(Hv)).astype(np.float32)) for _ in range(d.n_layers)]
+            ae.attach_vlm_kv(wk, wv, gn, Hv)
+            hid = torch.from_numpy(mk((d.batch, d.n_layers, d.n_prefix, Hv), 1.0).view(np.int16)).cuda()
+            for _ in range(3):
+                ae.set_prefix_hidden(hid, d.n_prefix, sdev, stream)
+            torch.cuda.synchronize()
+            reps = 20
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                ae.set_prefix_hidden(hid, d.n_prefix, sdev, stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms_p = a.elapsed_time(b) / reps
+            flops = 2.0 * d.batch * d.n_prefix * Hv * 2 * d.kd * d.n_layers
+            try:
+                with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                    tpk = float(json.load(f)["bf16_tflops"])
+            except Exception:
+                tpk = 1590.0
+            tf = flops / (ms_p * 1e-3) / 1e12
+            line["prefix_kv_producer"] = {
+                "ms_per_prefix": round(ms_p, 4), "tflops": round(tf, 2), "peak_tflops": tpk,
+                "frac": round(tf / tpk, 4), "bound": "tensor",
+                "shape": f"{d.n_layers} layers x [{d.batch * d.n_prefix} tokens x {Hv}] x [{Hv} x {2 * d.kd}] (K and V)",
+                "note": "operands are hi/lo bf16 pairs (2x the MMA work of plain bf16); FLOPs counted once"}
+            ae.set_prefix(kdev, vdev, d.n_prefix, sdev, on_device=True, stream=stream)
         # per-kernel timing through the bench hook: PDL-chained launches over successive layers
         L = d.n_layers
         count = 4 * L

@@ -17,7 +17,8 @@ __all__ = [
     "lib", "VlaAeDims", "VlaAeWeights", "VlaAeTrace", "VlaAeError", "ActionExpert",
     "vla_ae_create", "vla_ae_set_prefix", "vla_ae_denoise", "vla_ae_denoise_host", "vla_ae_status",
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
-    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "vla_ae_denoise_sched", "vla_ae_set_prefix_next", "vla_ae_denoise_stale", "BF16", "FP8_E4M3", "INT8", "INT4_G128", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
+    "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "vla_ae_denoise_sched", "vla_ae_set_prefix_next", "vla_ae_denoise_stale", "vla_ae_attach_vlm_kv", "vla_ae_set_prefix_hidden",
+    "vla_ae_debug_prefix_kv", "VlaAeVlmKvWeights", "BF16", "FP8_E4M3", "INT8", "INT4_G128", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
     "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES", "Q_ENGINE", "ENGINE_PER_OP", "ENGINE_PERSISTENT",
 ]
 
@@ -50,6 +51,11 @@ class VlaAeWeights(ctypes.Structure):
                 ("w_fada", _P), ("b_fada", _P), ("w_out", _P), ("b_out", _P), ("on_device", ctypes.c_int)]
 
 
+class VlaAeVlmKvWeights(ctypes.Structure):
+    _fields_ = [("hidden_vlm", ctypes.c_int), ("rms_eps", ctypes.c_float), ("on_device", ctypes.c_int),
+                ("wk", _PP), ("wv", _PP), ("gain", _PP)]
+
+
 class VlaAeTrace(ctypes.Structure):
     _fields_ = [(n, _P) for n in ("q", "k", "v", "o", "h_attn", "m")]
 
@@ -80,6 +86,9 @@ vla_ae_debug_weight = _sig("vla_ae_debug_weight", ctypes.c_int, _H, ctypes.c_int
 vla_ae_bench_op = _sig("vla_ae_bench_op", ctypes.c_int, _H, ctypes.c_int, ctypes.c_int, ctypes.c_int, _P)
 vla_ae_debug_wait_probe = _sig("vla_ae_debug_wait_probe", ctypes.c_int, _H, ctypes.c_uint)
 vla_ae_set_engine = _sig("vla_ae_set_engine", ctypes.c_int, _H, ctypes.c_int)
+vla_ae_attach_vlm_kv = _sig("vla_ae_attach_vlm_kv", ctypes.c_int, _H, ctypes.POINTER(VlaAeVlmKvWeights))
+vla_ae_set_prefix_hidden = _sig("vla_ae_set_prefix_hidden", ctypes.c_int, _H, _P, ctypes.c_int, _P, _P)
+vla_ae_debug_prefix_kv = _sig("vla_ae_debug_prefix_kv", ctypes.c_int, _H, ctypes.c_int, _P, _P)
 vla_ae_set_prefix_next = _sig("vla_ae_set_prefix_next", ctypes.c_int, _H, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P)
 vla_ae_denoise_stale = _sig("vla_ae_denoise_stale", ctypes.c_int, _H, _P, ctypes.c_int, ctypes.c_int, _P, _P)
 vla_ae_denoise_sched = _sig("vla_ae_denoise_sched", ctypes.c_int, _H, _P, ctypes.POINTER(ctypes.c_float),
@@ -162,6 +171,22 @@ class ActionExpert:
     def denoise(self, noise, steps: int, out, stream=None):
         _check(vla_ae_denoise(self.handle, _ptr(noise), int(steps), _ptr(out), _stream_ptr(stream)),
                "vla_ae_denoise")
+
+    def attach_vlm_kv(self, wk: Sequence, wv: Sequence, gain: Sequence, hidden_vlm: int, rms_eps: float = 1e-6):
+        """Backbone K/V projections per layer (host bf16 arrays; see vla_ae_attach_vlm_kv)."""
+        arr = lambda xs: (ctypes.c_void_p * len(xs))(*[_ptr(x) for x in xs])
+        keep = (arr(wk), arr(wv), arr(gain))
+        w = VlaAeVlmKvWeights(int(hidden_vlm), float(rms_eps), 0,
+                              ctypes.cast(keep[0], _PP), ctypes.cast(keep[1], _PP), ctypes.cast(keep[2], _PP))
+        _check(vla_ae_attach_vlm_kv(self.handle, ctypes.byref(w)), "vla_ae_attach_vlm_kv")
+
+    def set_prefix_hidden(self, hidden, n_prefix: int, state=None, stream=None):
+        """The current prefix from device bf16 hidden states [B][L][P][Hv] (see vla_ae_set_prefix_hidden)."""
+        _check(vla_ae_set_prefix_hidden(self.handle, _ptr(hidden), int(n_prefix), _ptr(state), _stream_ptr(stream)),
+               "vla_ae_set_prefix_hidden")
+
+    def debug_prefix_kv(self, layer: int, k, v):
+        _check(vla_ae_debug_prefix_kv(self.handle, int(layer), _ptr(k), _ptr(v)), "vla_ae_debug_prefix_kv")
 
     def set_prefix_next(self, k, v, n_prefix: int, state=None, on_device: bool = False, stream=None):
         """Lay out the next cycle's prefix (see vla_ae_set_prefix_next)."""

@@ -295,6 +295,100 @@ __global__ void quant_int4_kernel(const __nv_bfloat16* const* __restrict__ rows,
   }
 }
 
+// Prefix K/V producer operand of layer l: per prefix token row t = b * P + j, the sum of squares
+// of h (one part) and the hi/lo bf16 tiles of h * gain, 8 inputs (one 16-byte chunk of each tile)
+// per thread.  hidden [B][L][P][Hv] bf16, Hv % 8 == 0.  Launched chained after the previous
+// layer's GEMM: the operand is overwritten only after that GEMM has finished reading it.
+__global__ void prefix_operand_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ gain,
+                                      int L, int l, int P, int Hv, float* ss, __nv_bfloat16* tiles, int NT, int KB) {
+  pdl_trigger();
+  const int t = blockIdx.x, b = t / P, j = t % P;
+  const __nv_bfloat16* h = hidden + (((size_t)b * L + l) * P + j) * Hv;
+  __shared__ float red[32];
+  float acc = 0.f;
+  uint4 raw[2];
+  float4 g[4];
+  const int nch = Hv / 8;
+  // static inputs first, then wait for the previous kernel of the stream
+  int c = threadIdx.x;
+  const bool two = c + (int)blockDim.x < nch;
+  if (c < nch) {
+    raw[0] = __ldg(reinterpret_cast<const uint4*>(h) + c);
+    g[0] = __ldg(reinterpret_cast<const float4*>(gain) + 2 * c);
+    g[1] = __ldg(reinterpret_cast<const float4*>(gain) + 2 * c + 1);
+  }
+  if (two) {
+    raw[1] = __ldg(reinterpret_cast<const uint4*>(h) + c + blockDim.x);
+    g[2] = __ldg(reinterpret_cast<const float4*>(gain) + 2 * (c + blockDim.x));
+    g[3] = __ldg(reinterpret_cast<const float4*>(gain) + 2 * (c + blockDim.x) + 1);
+  }
+  pdl_wait();
+  for (int rep = 0; rep < 2 && c < nch; ++rep, c += blockDim.x) {
+    const uint4 r = rep == 0 ? raw[0] : raw[1];
+    const float gg[8] = {rep == 0 ? g[0].x : g[2].x, rep == 0 ? g[0].y : g[2].y, rep == 0 ? g[0].z : g[2].z,
+                         rep == 0 ? g[0].w : g[2].w, rep == 0 ? g[1].x : g[3].x, rep == 0 ? g[1].y : g[3].y,
+                         rep == 0 ? g[1].z : g[3].z, rep == 0 ? g[1].w : g[3].w};
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w[q]);
+      const float x0 = __low2float(pr), x1 = __high2float(pr);
+      acc = fmaf(x0, x0, acc);
+      acc = fmaf(x1, x1, acc);
+      const float v0 = x0 * gg[2 * q], v1 = x1 * gg[2 * q + 1];
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(v0, v1);
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v0 - __low2float(hi), v1 - __high2float(hi));
+      hw[q] = *reinterpret_cast<const uint32_t*>(&hi);
+      lw[q] = *reinterpret_cast<const uint32_t*>(&lo);
+    }
+    const size_t off = operand_offset(t, c * 8, NT, KB);
+    *reinterpret_cast<uint4*>(tiles + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(tiles + off + (size_t)NT * 64) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+  for (; c < nch; c += blockDim.x) {   // widths past 2 x blockDim x 8
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(h) + c);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&w[q]);
+      const float x0 = __low2float(pr), x1 = __high2float(pr);
+      acc = fmaf(x0, x0, acc);
+      acc = fmaf(x1, x1, acc);
+      const float v0 = x0 * __ldg(gain + c * 8 + 2 * q), v1 = x1 * __ldg(gain + c * 8 + 2 * q + 1);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(v0, v1);
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v0 - __low2float(hi), v1 - __high2float(hi));
+      hw[q] = *reinterpret_cast<const uint32_t*>(&hi);
+      lw[q] = *reinterpret_cast<const uint32_t*>(&lo);
+    }
+    const size_t off = operand_offset(t, c * 8, NT, KB);
+    *reinterpret_cast<uint4*>(tiles + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(tiles + off + (size_t)NT * 64) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s2 = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s2 += red[w];
+    ss[t] = s2;
+  }
+}
+
+// prefix rows of one layer's caches -> fp32 k, v [B][P][nkv][hd]
+__global__ void prefix_kv_readback_kernel(const __nv_bfloat16* kc, const __nv_bfloat16* vct, float* k, float* v, int B,
+                                          int P, int nkv, int hd, int Lpad) {
+  const size_t n = (size_t)B * P * nkv * hd;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
+    const int d = e % hd, g = (e / hd) % nkv, j = (e / ((size_t)hd * nkv)) % P, b = e / ((size_t)hd * nkv * P);
+    const size_t cache = (size_t)b * nkv + g;
+    k[e] = __bfloat162float(kc[(cache * Lpad + j) * hd + d]);
+    v[e] = __bfloat162float(vct[(cache * hd + d) * Lpad + j]);
+  }
+}
+
 // ---------------------------------------------------------------- prefix layout (set_prefix)
 // user K, V: [B][L][P][nkv][hd]  ->  K cache [L][B][nkv][Lpad][hd], V^T cache [L][B][nkv][hd][Lpad]
 __global__ void prefix_layout_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,

@@ -119,6 +119,15 @@ struct vla_ae {
   bool next_pending = false;
   cudaEvent_t next_ready = nullptr;
   int attn_P = -1;            // prefix length the per-op attention plan was made for
+  // prefix K/V producer (vla_ae_attach_vlm_kv)
+  bool vlm = false;
+  int Hv = 0, NTp = 0, Ntp = 0;
+  float vlm_eps = 1e-6f;
+  OpPlan pkv;                 // the K/V GEMM over the prefix tokens (bf16)
+  uint8_t* wpack_vlm = nullptr;
+  float* vlm_gain = nullptr;  // [L][Hv]
+  __nv_bfloat16* act_p = nullptr;   // operand tiles [Ntp][KBp][2][NTp][64]
+  float *ss_p = nullptr, *rope_p = nullptr, *zeros_p = nullptr;
   cudaStream_t cap = nullptr;
   std::map<std::vector<double>, StepTables> tables;   // keyed by the time grid
 
@@ -170,6 +179,23 @@ cudaError_t launch(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
   cfg.attrs = attrs;
   cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, arg);
+}
+
+// Plain-argument kernel launch, optionally chained by programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_args(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                        Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at;
+  at.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &at;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // One CTA per SM for the whole launch: the cooperative attribute makes the launch fail instead of
@@ -274,17 +300,18 @@ bool cluster_fits(GemmKernel kern, const OpPlan& p, int Nt, bool one_wave) {
 
 // Choose m-tiles per CTA and the split so that one wave of CTAs covers the GPU with the
 // fewest weight tiles per CTA, inside the shared-memory budget that keeps two CTAs per SM.
-int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
-  const bool fp8 = H->fp8;
+// Split / m-group / ring plan of one GEMM over Nt token tiles of NT rows with weight format wq.
+int plan_gemm_shape(vla_ae* H, OpPlan& out, OpId id, int O, int K, int NT, int Nt, int wq) {
+  const bool fp8 = wq != 0;
   OpPlan base;
   base.O = O;
   base.K = K;
   base.Mt = ceil_div(O, 128);
   base.KB = ceil_div(K, 64);
-  const int kpt = wq_kpt(H->wq);
+  const int kpt = wq_kpt(wq);
   base.KBt = ceil_div(K, 64 * kpt);
   base.wbytes = (size_t)base.Mt * base.KBt * kTileBytes;
-  GemmKernel kern = gemm_kernel_for(id, H->wq);
+  GemmKernel kern = gemm_kernel_for(id, wq);
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
   CK(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem));
   // every kernel of the loop asks for the same (maximum) shared-memory carveout, so SMs never
@@ -297,10 +324,10 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
   for (int pass = 0; pass < 2 && !found; ++pass) {      // pass 1 allows more than one wave
     for (int mpc : {1, 2, 4}) {
       // TMEM: half of it (room for a second CTA per SM), or all of it in the fallback pass
-      if (mpc > base.Mt || mpc * 2 * H->NT > (pass == 0 ? 256 : 512)) continue;
+      if (mpc > base.Mt || mpc * 2 * NT > (pass == 0 ? 256 : 512)) continue;
       const int mg = ceil_div(base.Mt, mpc);
       for (int S = 1; S <= std::min(16, base.KBt); ++S) {
-        const int ctas = mg * S * H->Nt;
+        const int ctas = mg * S * Nt;
         if (pass == 0 && ctas > H->num_sms) continue;   // pass 1: several waves (large batches)
         OpPlan p = base;
         p.mpc = mpc;
@@ -308,11 +335,11 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
         const int tiles = mpc * ceil_div(base.KBt, S);
         // deepest ring inside the budget (at least 2 stages when there is more than one tile)
         p.stages = 1;
-        gemm_layout(p, H->NT, kpt);
+        gemm_layout(p, NT, kpt);
         for (int st = 2; st <= std::min(tiles, 8); ++st) {
           OpPlan t = p;
           t.stages = st;
-          gemm_layout(t, H->NT, kpt);
+          gemm_layout(t, NT, kpt);
           if (t.smem > (fp8 ? kMaxDynSmem : budget) && p.stages >= 2) break;
           if (t.smem > kMaxDynSmem) break;
           p = t;
@@ -322,7 +349,7 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
         // lexicographic: inside budget, fewest tiles per CTA, smallest split, fewest m-tiles per CTA
         const long key = (long)over * 1000000 + (long)tiles * 1000 + S * 10 + mpc;
         if (found && key >= best_key) continue;
-        if (!cluster_fits(kern, p, H->Nt, pass == 0)) continue;
+        if (!cluster_fits(kern, p, Nt, pass == 0)) continue;
         best = p;
         best_key = key;
         found = true;
@@ -332,6 +359,10 @@ int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
   if (!found) return VLA_AE_EUNSUPPORTED;
   out = best;
   return VLA_AE_OK;
+}
+
+int plan_gemm(vla_ae* H, OpPlan& out, OpId id, int O, int K) {
+  return plan_gemm_shape(H, out, id, O, K, H->NT, H->Nt, H->wq);
 }
 
 // Which source matrix row feeds packed row `pr` of op `id` (matrix: 0 q,1 k,2 v,3 o,4 g,5 u,6 d; -1 pad).
@@ -1280,6 +1311,145 @@ int vla_ae_set_prefix(vla_ae_t H, const void* k, const void* v, int n_prefix, co
   int rc = write_prefix(H, H->front, k, v, n_prefix, state, on_device, reinterpret_cast<cudaStream_t>(stream));
   if (rc) return rc;
   return use_slot(H, H->front);
+}
+
+int vla_ae_attach_vlm_kv(vla_ae_t H, const vla_ae_vlm_kv_weights* w) {
+  if (!H || !w || w->hidden_vlm < 8 || w->hidden_vlm % 8 != 0 || !(w->rms_eps >= 0.f) || !w->wk || !w->wv || !w->gain)
+    return VLA_AE_EINVAL;
+  if (H->vlm) return VLA_AE_EINVAL;   // once per handle
+  const vla_ae_dims& d = H->d;
+  const int Hv = w->hidden_vlm, kd = H->kd, L = d.n_layers;
+  // token tiling of the prefix rows (as for the action tokens: <= 128 rows per tile)
+  const int ntok = d.batch * std::max(1, d.max_prefix);
+  H->Ntp = ceil_div(ntok, 128);
+  H->NTp = (int)align_up((size_t)ceil_div(ntok, H->Ntp), 32);
+  int rc;
+  if ((rc = plan_gemm_shape(H, H->pkv, OP_QKV, 2 * kd, Hv, H->NTp, H->Ntp, 0))) return rc;
+  OpPlan& pk = H->pkv;
+  if ((rc = H->alloc(&H->wpack_vlm, (size_t)L * pk.wbytes))) return rc;
+  if ((rc = H->alloc(&H->vlm_gain, (size_t)L * Hv * 4))) return rc;
+  if ((rc = H->alloc(&H->act_p, (size_t)H->Ntp * pk.KB * 2 * H->NTp * 64 * 2))) return rc;
+  if ((rc = H->alloc(&H->ss_p, (size_t)H->Ntp * H->NTp * 4))) return rc;
+  if ((rc = H->alloc(&H->rope_p, (size_t)std::max(1, d.max_prefix) * (d.head_dim / 2) * 8))) return rc;
+  if ((rc = H->alloc(&H->zeros_p, (size_t)pk.Mt * 128 * 4))) return rc;
+  // pack per layer: rows [0, kd) k with rotary pairs adjacent (as the QKV GEMM's k rows), then v
+  const int hd = d.head_dim, half = hd / 2;
+  __nv_bfloat16 *sk = nullptr, *sv = nullptr, *sg = nullptr;
+  CK(cudaMalloc(&sk, (size_t)kd * Hv * 2));
+  CK(cudaMalloc(&sv, (size_t)kd * Hv * 2));
+  CK(cudaMalloc(&sg, (size_t)Hv * 2));
+  const __nv_bfloat16** rowptr_dev = nullptr;
+  CK(cudaMalloc(&rowptr_dev, (size_t)pk.Mt * 128 * sizeof(void*)));
+  std::vector<const __nv_bfloat16*> rows((size_t)pk.Mt * 128, nullptr);
+  const cudaMemcpyKind kind = w->on_device ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+  for (int l = 0; l < L; ++l) {
+    if (!w->wk[l] || !w->wv[l] || !w->gain[l]) return VLA_AE_EINVAL;
+    CK(cudaMemcpy(sk, w->wk[l], (size_t)kd * Hv * 2, kind));
+    CK(cudaMemcpy(sv, w->wv[l], (size_t)kd * Hv * 2, kind));
+    CK(cudaMemcpy(sg, w->gain[l], (size_t)Hv * 2, kind));
+    for (int pr = 0; pr < pk.Mt * 128; ++pr) {
+      const __nv_bfloat16* src = nullptr;
+      if (pr < kd) {
+        const int head = pr / hd, i = (pr % hd) / 2;
+        src = sk + (size_t)(head * hd + i + (pr & 1) * half) * Hv;
+      } else if (pr < 2 * kd) {
+        src = sv + (size_t)(pr - kd) * Hv;
+      }
+      rows[pr] = src;
+    }
+    CK(cudaMemcpy(rowptr_dev, rows.data(), rows.size() * sizeof(void*), cudaMemcpyHostToDevice));
+    pack_bf16_kernel<<<1024, 256>>>(rowptr_dev, Hv, pk.Mt, pk.KB, H->wpack_vlm + (size_t)l * pk.wbytes);
+    bf16_to_f32_kernel<<<ceil_div(Hv, 256), 256>>>(sg, H->vlm_gain + (size_t)l * Hv, (size_t)Hv);
+    CK(cudaGetLastError());
+    CK(cudaDeviceSynchronize());   // the staging buffers are reused
+  }
+  cudaFree(sk);
+  cudaFree(sv);
+  cudaFree(sg);
+  cudaFree(rowptr_dev);
+  H->Hv = Hv;
+  H->vlm_eps = w->rms_eps;
+  H->vlm = true;
+  return VLA_AE_OK;
+}
+
+int vla_ae_set_prefix_hidden(vla_ae_t H, const void* hidden, int n_prefix, const void* state, void* stream) {
+  if (!H || !H->vlm || !hidden || n_prefix < 1 || n_prefix > H->d.max_prefix) return VLA_AE_EINVAL;
+  if (H->d.has_state_token && !state) return VLA_AE_EINVAL;
+  const vla_ae_dims& d = H->d;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const OpPlan& pk = H->pkv;
+  const int ntok = d.batch * n_prefix, Nt = ceil_div(ntok, H->NTp);
+  PrefixSlot& sl = H->slot[H->front];
+  const size_t cache_layer = (size_t)d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+  rope_table_kernel<<<ceil_div(n_prefix * d.head_dim / 2, 256), 256, 0, st>>>(reinterpret_cast<float2*>(H->rope_p),
+                                                                              n_prefix, 0, d.head_dim,
+                                                                              (double)d.rope_theta);
+  for (int l = 0; l < d.n_layers; ++l) {
+    CK(launch_args(prefix_operand_kernel, dim3(ntok), dim3(128), 0, st, l > 0,
+                   reinterpret_cast<const __nv_bfloat16*>(hidden), (const float*)(H->vlm_gain + (size_t)l * H->Hv),
+                   (int)d.n_layers, l, n_prefix, H->Hv, H->ss_p, H->act_p, H->NTp, pk.KB));
+    GemmParams g{};
+    g.w = H->wpack_vlm + (size_t)l * pk.wbytes;
+    g.Mt = pk.Mt;
+    g.mpc = pk.mpc;
+    g.KBt = pk.KBt;
+    g.K = pk.K;
+    g.S = pk.S;
+    g.stages = pk.stages;
+    g.Ntok = ntok;
+    g.NT = H->NTp;
+    g.KB = pk.KB;
+    g.O = pk.O;
+    g.act = H->act_p;
+    g.ss = H->ss_p;
+    g.ss_parts = 1;
+    g.cshift = H->zeros_p;
+    g.inv_h = 1.0f / (float)H->Hv;
+    g.eps = H->vlm_eps;
+    g.kc = sl.kc + (size_t)l * cache_layer;
+    g.vct = sl.vct + (size_t)l * cache_layer;
+    g.rope = H->rope_p;
+    g.nq = 0;   // K and V rows only
+    g.nkv = d.n_kv_heads;
+    g.hd = d.head_dim;
+    g.Ts = n_prefix;   // token t -> sample t / P, position t % P
+    g.P = 0;
+    g.Lpad = H->Lpad;
+    g.status = H->status;
+    g.spr = 1;
+    g.off_b = pk.off_b;
+    g.off_conv = pk.off_conv;
+    g.off_bar = pk.off_bar;
+    g.off_misc = pk.off_misc;
+    g.off_vec = pk.off_vec;
+    g.smem_bytes = pk.smem;
+    CK(launch(gemm_kernel_for(OP_QKV, 0), dim3(pk.S, ceil_div(pk.Mt, pk.mpc), Nt), dim3(kGemmThreads), pk.smem, st,
+              pk.S, true, g));
+  }
+  // state token and the RoPE table of the self tokens at positions n_prefix + j
+  if (d.has_state_token) {
+    CK(cudaMemcpyAsync(H->state_stage, state, (size_t)d.batch * d.action_dim * 2, cudaMemcpyDeviceToDevice, st));
+    state_proj_kernel<<<dim3(ceil_div(d.hidden, 256), d.batch), 256, 0, st>>>(H->w_st, H->b_st, H->state_stage,
+                                                                               sl.h_state0, d.hidden, d.action_dim);
+  }
+  rope_table_kernel<<<ceil_div(H->Ts * d.head_dim / 2, 256), 256, 0, st>>>(reinterpret_cast<float2*>(sl.rope), H->Ts,
+                                                                           n_prefix, d.head_dim, (double)d.rope_theta);
+  CK(cudaGetLastError());
+  sl.n_prefix = n_prefix;
+  return use_slot(H, H->front);
+}
+
+int vla_ae_debug_prefix_kv(vla_ae_t H, int layer, float* k, float* v) {
+  if (!H || !k || !v || layer < 0 || layer >= H->d.n_layers) return VLA_AE_EINVAL;
+  if (H->n_prefix < 0) return VLA_AE_ENOPREFIX;
+  const vla_ae_dims& d = H->d;
+  const size_t cache_layer = (size_t)d.batch * d.n_kv_heads * H->Lpad * d.head_dim;
+  prefix_kv_readback_kernel<<<64, 256, 0, H->cap>>>(H->kc + layer * cache_layer, H->vct + layer * cache_layer, k, v,
+                                                    d.batch, H->n_prefix, d.n_kv_heads, d.head_dim, H->Lpad);
+  CK(cudaGetLastError());
+  CK(cudaStreamSynchronize(H->cap));
+  return VLA_AE_OK;
 }
 
 int vla_ae_set_prefix_next(vla_ae_t H, const void* k, const void* v, int n_prefix, const void* state, int on_device,

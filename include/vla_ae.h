@@ -138,6 +138,36 @@ int vla_ae_set_prefix_static(vla_ae_t h, const void *k, const void *v, int n_pre
  * `stream`.  Errors: EINVAL, ENOPREFIX, ECUDA. */
 int vla_ae_denoise(vla_ae_t h, const void *noise, int steps, float *out, void *stream);
 
+/* ------------------------------------------------------------------ prefix K/V producer
+ * The VLM side of the cached prefix ("AI Infra如何优化VLA", section 算子开发: the backbone's pre-norm
+ * RMSNorm and the half-split RoPE of the prefill): for every layer l the hidden states h_l of the
+ * P prefix tokens become x = RMSNorm(h_l) * gain_l, K_l = RoPE(x Wk_l^T) at positions 0..P-1 and
+ * V_l = x Wv_l^T, written straight into the loop's caches (the expert attends to the backbone's
+ * K/V, so its kv heads are the backbone's).  bf16 weights; the GEMM is the QKV kernel without q
+ * heads, the RMSNorm scale applied by linearity.
+ *
+ * vla_ae_attach_vlm_kv: copy and pack the backbone's per-layer K/V projections.
+ *   hidden_vlm  Hv, the backbone's width (% 8 == 0);   rms_eps  its RMSNorm epsilon;
+ *   wk, wv      [L] arrays of bf16 [nkv*hd][Hv];  gain  [L] arrays of bf16 [Hv];
+ *   on_device   1: device pointers (16-byte aligned), 0: host.
+ * Synchronous.  Errors: EINVAL, ENOMEM, ECUDA, EUNSUPPORTED.
+ *
+ * vla_ae_set_prefix_hidden: the current prefix from device bf16 hidden states [B][L][P][Hv]
+ * (n_prefix <= max_prefix) and the state token as in vla_ae_set_prefix.  Asynchronous on
+ * `stream`.  Errors: EINVAL (also before vla_ae_attach_vlm_kv), ECUDA. */
+typedef struct {
+  int hidden_vlm;
+  float rms_eps;
+  int on_device;
+  const void *const *wk, *const *wv, *const *gain;
+} vla_ae_vlm_kv_weights;
+int vla_ae_attach_vlm_kv(vla_ae_t h, const vla_ae_vlm_kv_weights *w);
+int vla_ae_set_prefix_hidden(vla_ae_t h, const void *hidden, int n_prefix, const void *state, void *stream);
+
+/* Test hook: the current prefix's cached rows of layer `layer` as device fp32 k, v [B][P][nkv][hd]
+ * (K after RoPE).  Synchronous.  Errors: EINVAL, ENOPREFIX, ECUDA. */
+int vla_ae_debug_prefix_kv(vla_ae_t h, int layer, float *k, float *v);
+
 /* ------------------------------------------------------------------ stale-prefix overlap
  * V-AEFusion ("跨XPU平台表征视觉-语言-动作模型" section 5.3): the first denoising steps of a control
  * cycle run on the previous cycle's prefix while the VLM computes the new one on another stream;

@@ -103,6 +103,9 @@ def test_null_arguments(fm):
     assert fm.vla_ae_set_engine(None, fm.ENGINE_PER_OP) == fm.EINVAL
     assert fm.vla_ae_set_prefix_next(None, None, None, 0, None, 0, None) == fm.EINVAL
     assert fm.vla_ae_denoise_stale(None, None, 4, 2, None, None) == fm.EINVAL
+    assert fm.vla_ae_attach_vlm_kv(None, None) == fm.EINVAL
+    assert fm.vla_ae_set_prefix_hidden(None, None, 1, None, None) == fm.EINVAL
+    assert fm.vla_ae_debug_prefix_kv(None, 0, None, None) == fm.EINVAL
     fm.vla_ae_destroy(None)   # no-op
 
 

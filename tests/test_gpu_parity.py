@@ -286,6 +286,59 @@ def test_stale_prefix_overlap(name, eng):
         c.ae.set_prefix(cur[1], cur[2], cur[3], cur[0])   # leave the shared case as it was
 
 
+def _vlm_weights(d, Hv, seed):
+    """Synthetic backbone K/V projections (N(0, 0.02)) and RMSNorm gains (1 + N(0, 0.1)), bf16 bits."""
+    from synth import f32_to_bf16_bits
+    rng = np.random.default_rng(seed)
+    wk = [f32_to_bf16_bits((rng.standard_normal((d.kd, Hv)) * 0.02).astype(np.float32)) for _ in range(d.n_layers)]
+    wv = [f32_to_bf16_bits((rng.standard_normal((d.kd, Hv)) * 0.02).astype(np.float32)) for _ in range(d.n_layers)]
+    g = [f32_to_bf16_bits((1.0 + 0.1 * rng.standard_normal(Hv)).astype(np.float32)) for _ in range(d.n_layers)]
+    return wk, wv, g
+
+
+@pytest.mark.parametrize("name,Hv", [("tiny", 320), ("ragged", 136)])
+def test_prefix_kv_producer(name, Hv):
+    """Backbone hidden states -> cached prefix K/V (RMSNorm, projection, RoPE at 0..P-1), then the loop."""
+    import flow_matching_action_euler_b200 as fm
+    from synth import abi_dims, f32_to_bf16_bits, generate_inputs, generate_weights
+    d = RAGGED if name == "ragged" else config(name)
+    P = d.n_prefix
+    w = generate_weights(d, 0)
+    x = generate_inputs(d, 0)
+    wk, wv, g = _vlm_weights(d, Hv, 7)
+    rng = np.random.default_rng(8)
+    hid = f32_to_bf16_bits(rng.standard_normal((d.batch, d.n_layers, P, Hv)).astype(np.float32))
+    ae = fm.ActionExpert(abi_dims(d), w)
+    try:
+        ae.attach_vlm_kv(wk, wv, g, Hv)
+        ae.set_prefix_hidden(torch.from_numpy(hid.view(np.int16)).cuda(), P,
+                             torch.from_numpy(x["state"].view(np.int16)).cuda() if d.has_state_token else None)
+        torch.cuda.synchronize()
+        kref = np.zeros((d.batch, d.n_layers, P, d.n_kv_heads, d.head_dim))
+        vref = np.zeros_like(kref)
+        f = oracle.bf16_to_f64
+        for b in range(d.batch):
+            for l in range(d.n_layers):
+                kref[b, l], vref[b, l] = oracle.prefix_kv(f(hid[b, l]), f(wk[l]), f(wv[l]), f(g[l]), d.n_kv_heads)
+        for l in range(d.n_layers):
+            kg = torch.empty((d.batch, P, d.n_kv_heads, d.head_dim), device="cuda")
+            vg = torch.empty_like(kg)
+            ae.debug_prefix_kv(l, kg, vg)
+            # the caches hold bf16: compare at bf16 resolution
+            assert rel_err(kg.cpu().numpy(), kref[:, l]) <= 1e-2, l
+            assert rel_err(vg.cpu().numpy(), vref[:, l]) <= 1e-2, l
+        # the whole loop on that prefix against the oracle loop on the oracle's K/V (bf16-rounded)
+        kb, vb = f32_to_bf16_bits(kref.astype(np.float32)), f32_to_bf16_bits(vref.astype(np.float32))
+        noise = torch.from_numpy(x["noise"].view(np.int16)).cuda()
+        out = torch.empty((d.batch, d.n_action_tokens, d.action_dim), dtype=torch.float32, device="cuda")
+        ae.denoise(noise, d.steps, out)
+        torch.cuda.synchronize()
+        ref = oracle.denoise_batch(w, {**x, "k": kb, "v": vb}, d)
+        assert rel_err(out.cpu().numpy(), ref) <= FINAL_TOL
+    finally:
+        ae.close()
+
+
 def test_denoise_is_deterministic_across_replays():
     c = case("tiny")
     a = c.denoise()
