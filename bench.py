@@ -358,7 +358,7 @@ def run_native(args):
         "vs_baseline": None, "dtype": {"bf16": "bf16", "fp8_e4m3": "e4m3 weights x bf16 activations",
                   "int8": "int8 weights x bf16 activations",
                   "int4_g128": "int4 weights (groups of 128) x bf16 activations"}[d.wtype],
-        "data": "synthetic", "config": {**workload_config(d, args), "engine": engine},
+        "data": "synthetic", "config": workload_config(d, args), "engine": engine,
         "ms_per_loop": round(ms, 5),
         "actions_per_s": round(world * d.batch * d.n_action_tokens * 1000.0 / ms, 1),
         "chunks_per_s": round(world * d.batch * 1000.0 / ms, 2),
