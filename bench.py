@@ -50,8 +50,9 @@ def parse_args():
     ap.add_argument("--euler-steps", type=int, default=None, help="Euler steps per loop (default: workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip e2e / per-kernel timing (profiling runs)")
-    ap.add_argument("--engine", choices=("default", "per_op", "persistent"), default="default",
-                    help="layer engine: one kernel per op (the library default) or one persistent kernel per step")
+    ap.add_argument("--engine", choices=("auto", "per_op", "persistent"), default="auto",
+                    help="layer engine: auto (the library times both on the first loop and keeps the "
+                         "faster), one kernel per op, or one persistent kernel per step")
     return ap.parse_args()
 
 
@@ -306,9 +307,8 @@ def run_native(args):
     vdev = torch.from_numpy(x["v"].view(np.int16)).cuda()
     sdev = torch.from_numpy(x["state"].view(np.int16)).cuda() if d.has_state_token else None
     ae.set_prefix(kdev, vdev, d.n_prefix, sdev, on_device=True, stream=stream)
-    if args.engine != "default":
-        ae.set_engine(fm.ENGINE_PERSISTENT if args.engine == "persistent" else fm.ENGINE_PER_OP)
-    engine = "persistent" if ae.engine == fm.ENGINE_PERSISTENT else "per_op"
+    ae.set_engine({"auto": fm.ENGINE_AUTO, "per_op": fm.ENGINE_PER_OP,
+                   "persistent": fm.ENGINE_PERSISTENT}[args.engine])
     noise = torch.from_numpy(x["noise"].view(np.int16)).cuda()
     out = torch.empty((d.batch, d.n_action_tokens, d.action_dim), dtype=torch.float32, device="cuda")
     N = d.steps
@@ -317,8 +317,9 @@ def run_native(args):
         if world > 1:
             dist.barrier()
 
-    ae.denoise(noise, N, out, stream)          # first call: adaLN table + graph capture
+    ae.denoise(noise, N, out, stream)          # first call: adaLN table + graph capture (auto: both engines timed)
     torch.cuda.synchronize()
+    engine = "persistent" if ae.engine == fm.ENGINE_PERSISTENT else "per_op"
     for _ in range(max(args.warmup, 3)):
         ae.denoise(noise, N, out, stream)
     torch.cuda.synchronize()
@@ -388,7 +389,8 @@ def run_native(args):
             torch.cuda.synchronize()
             engines[name] = {"ms_per_loop": round(a.elapsed_time(b) / reps, 4),
                              "kernels_per_loop": int(ae.query(fm.Q_KERNELS_PER_LOOP, N))}
-        ae.set_engine(fm.ENGINE_PERSISTENT if engine == "persistent" else fm.ENGINE_PER_OP)
+        ae.set_engine({"auto": fm.ENGINE_AUTO, "per_op": fm.ENGINE_PER_OP,
+                       "persistent": fm.ENGINE_PERSISTENT}[args.engine])
         line["engines"] = engines
         # prefix K/V producer (backbone RMSNorm + K/V projection + RoPE), synthetic backbone of
         # width 2048: the compute-bound neighbour stage, against the tensor-core peak

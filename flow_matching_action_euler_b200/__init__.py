@@ -19,12 +19,12 @@ __all__ = [
     "vla_ae_strerror", "vla_ae_destroy", "vla_ae_query", "vla_ae_debug_layer", "vla_ae_debug_velocity",
     "vla_ae_debug_weight", "vla_ae_bench_op", "vla_ae_set_prefix_static", "vla_ae_debug_wait_probe", "vla_ae_set_engine", "vla_ae_denoise_sched", "vla_ae_set_prefix_next", "vla_ae_denoise_stale", "vla_ae_attach_vlm_kv", "vla_ae_set_prefix_hidden",
     "vla_ae_debug_prefix_kv", "VlaAeVlmKvWeights", "BF16", "FP8_E4M3", "INT8", "INT4_G128", "Q_KERNELS_PER_LOOP", "Q_WEIGHT_BYTES", "Q_KV_BYTES",
-    "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES", "Q_ENGINE", "ENGINE_PER_OP", "ENGINE_PERSISTENT",
+    "Q_DEVICE_BYTES", "Q_SPLITS", "Q_OP_BYTES", "Q_ENGINE", "ENGINE_PER_OP", "ENGINE_PERSISTENT", "ENGINE_AUTO",
 ]
 
 BF16, FP8_E4M3, INT8, INT4_G128 = 0, 1, 2, 3
 Q_KERNELS_PER_LOOP, Q_WEIGHT_BYTES, Q_KV_BYTES, Q_DEVICE_BYTES, Q_SPLITS, Q_OP_BYTES, Q_ENGINE = 1, 2, 3, 4, 5, 6, 7
-ENGINE_PER_OP, ENGINE_PERSISTENT = 0, 1
+ENGINE_PER_OP, ENGINE_PERSISTENT, ENGINE_AUTO = 0, 1, 2
 OK, EINVAL, ENOMEM, ECUDA, ENOPREFIX, ETIMEOUT, EUNSUPPORTED = 0, -1, -2, -3, -4, -5, -6
 
 if not os.path.exists(LIB_PATH):
@@ -233,7 +233,8 @@ class ActionExpert:
         _check(vla_ae_debug_wait_probe(self.handle, int(attempts)), "vla_ae_debug_wait_probe")
 
     def set_engine(self, engine: int):
-        """ENGINE_PER_OP or ENGINE_PERSISTENT (raises EUNSUPPORTED where the latter is unavailable)."""
+        """ENGINE_PER_OP, ENGINE_PERSISTENT (raises EUNSUPPORTED where it is unavailable) or
+        ENGINE_AUTO (the first whole loop of a step count times both and keeps the faster)."""
         _check(vla_ae_set_engine(self.handle, engine), "vla_ae_set_engine")
 
     @property

@@ -204,11 +204,25 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
       const uint32_t bytes = (uint32_t)(kb1 - kb0) * 2u * NT * 128u;
       mbar_arrive_expect_tx(bfull, bytes);
       bulk_g2s(sB, p.act + ((size_t)nt * p.KB + kb0) * 2 * NT * 64, bytes, bfull, policy_evict_last());
-      for (int i = prefill; i < ntiles; ++i) {
-        const int s = i % p.stages;
-        if (!mbar_wait(&empty[s], ((i / p.stages) - 1) & 1, p.status, DEV_ERR_TIMEOUT_TMA)) break;
-        mbar_arrive_expect_tx(&full[s], kTileBytes);
-        bulk_g2s(sA + (size_t)s * kTileBytes, tile_src(i), kTileBytes, &full[s], pol);
+      if (prefill < ntiles) {
+        // tile i reuses stage i % stages once round i / stages - 1 of that stage was consumed
+        int s = 0, li = prefill % nkt;      // prefill == stages here, so tile `prefill` opens stage 0
+        uint32_t ph = 0;
+        const uint8_t* src = tile_src(prefill);
+        for (int i = prefill; i < ntiles; ++i) {
+          if (!mbar_wait(&empty[s], ph, p.status, DEV_ERR_TIMEOUT_TMA)) break;
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          bulk_g2s(sA + (size_t)s * kTileBytes, src, kTileBytes, &full[s], pol);
+          src += kTileBytes;
+          if (++li == nkt) {                // next m-tile: skip the k-tiles other ranks stream
+            li = 0;
+            src += (size_t)(p.KBt - nkt) * kTileBytes;
+          }
+          if (++s == p.stages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
       }
     }
     __syncwarp();
@@ -217,48 +231,63 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, stacked ? 2 * NT : NT);
       bool ok = mbar_wait(bfull, 0, p.status, DEV_ERR_TIMEOUT_TMA);
-      const uint32_t aBase = smem_u32(FP8 ? sC : sA), bBase = smem_u32(sB);
       const uint32_t bstride = (uint32_t)NT * 128u;   // bytes of one hi or lo tile
+      // descriptors of the first A stage and of the first operand k-block; a step of 16 bytes is
+      // one unit of the descriptor's start-address field (shared addresses stay below 256 KB, so
+      // adding offsets never carries out of that field).  This issue loop runs in one thread and
+      // sits on the kernel's critical path: no divisions, no descriptor rebuilds per tile.
+      const uint64_t a0 = sw128_desc(smem_u32(FP8 ? sC : sA)), b0 = sw128_desc(smem_u32(sB));
+      const uint64_t lo_off = bstride >> 4;           // hi tile -> lo tile
       // one (hi ++ lo) product per K step when stacked, else hi into cols [0,NT), lo into [NT,2NT)
-      auto mma_k = [&](uint32_t d_tmem, uint64_t ad, uint32_t bb, uint32_t acc) {
-        if (stacked) {
-          mma_bf16(d_tmem, ad, sw128_desc(bb), idesc, acc);
-        } else {
-          mma_bf16(d_tmem, ad, sw128_desc(bb), idesc, acc);
-          mma_bf16(d_tmem + (uint32_t)NT, ad, sw128_desc(bb + bstride), idesc, acc);
-        }
+      auto mma_k = [&](uint32_t d_tmem, uint64_t ad, uint64_t bd, uint32_t acc) {
+        mma_bf16(d_tmem, ad, bd, idesc, acc);
+        if (!stacked) mma_bf16(d_tmem + (uint32_t)NT, ad, bd + lo_off, idesc, acc);
       };
+      int s = 0, li = 0;                              // ring / conversion stage, local k-tile
+      uint32_t ph = 0;                                // its phase parity
+      uint32_t d_tmem = tmem_d;                       // accumulator of the current m-tile
       for (int i = 0; i < ntiles && ok; ++i) {
-        const int j = i / nkt, li = i % nkt;          // accumulator (m-tile), local k-tile
-        const uint32_t d_tmem = tmem_d + (uint32_t)(j * 2 * NT);
         if (!FP8) {
-          const int s = i % p.stages;
-          ok = mbar_wait(&full[s], (i / p.stages) & 1, p.status, DEV_ERR_TIMEOUT_TMA);
+          ok = mbar_wait(&full[s], ph, p.status, DEV_ERR_TIMEOUT_TMA);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t ad = a0 + (uint64_t)((uint32_t)s * (kTileBytes >> 4));
+          const uint64_t bd = b0 + (uint64_t)((uint32_t)li * 2u * lo_off);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_k(d_tmem, sw128_desc(aBase + s * kTileBytes + kk * 32), bBase + (uint32_t)li * 2u * bstride + kk * 32,
-                  (li | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk) mma_k(d_tmem, ad + 2 * kk, bd + 2 * kk, (li | kk) != 0);
           mma_commit(&empty[s]);
+          if (++s == p.stages) {
+            s = 0;
+            ph ^= 1u;
+          }
         } else {
-          const int c = i % kConvStages;
-          ok = mbar_wait(&cfull[c], (i / kConvStages) & 1, p.status, DEV_ERR_TIMEOUT_CONV);
+          ok = mbar_wait(&cfull[s], ph, p.status, DEV_ERR_TIMEOUT_CONV);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
           for (int half = 0; half < KPT; ++half) {
-            const int lkb = li * 2 + half;                      // local 64-wide k-block
+            const int lkb = li * KPT + half;                    // local 64-wide k-block
             if (kb0 + lkb >= kb1) break;                        // ragged K tail
+            const uint64_t ad = a0 + (uint64_t)((uint32_t)(s * KPT + half) * (kTileBytes >> 4));
+            const uint64_t bd = b0 + (uint64_t)((uint32_t)lkb * 2u * lo_off);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_k(d_tmem, sw128_desc(aBase + (c * KPT + half) * kTileBytes + kk * 32),
-                    bBase + (uint32_t)lkb * 2u * bstride + kk * 32, (lkb | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) mma_k(d_tmem, ad + 2 * kk, bd + 2 * kk, (lkb | kk) != 0);
           }
-          mma_commit(&cempty[c]);
+          mma_commit(&cempty[s]);
+          if (++s == kConvStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (++li == nkt) {
+          li = 0;
+          d_tmem += (uint32_t)(2 * NT);
         }
       }
       mma_commit(done);
+      // the epilogue warps learn that the accumulators are complete from the barrier below (one
+      // polling thread instead of four polling warps)
+      mbar_wait(done, 0, p.status, DEV_ERR_TIMEOUT_MMA);
     }
     __syncwarp();
   } else {
@@ -419,19 +448,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
   const int RST = NT + 4;                               // padded receive row (floats)
   float* recv = reinterpret_cast<float*>(sA);           // [S][rmax][RST]
   float vals[16];
-  if (warp >= 2) {
-    const bool ok = mbar_wait(done, 0, p.status, DEV_ERR_TIMEOUT_MMA);
-    tc_fence_after();
-    (void)ok;
-  }
+  // the MMA warp arrives only after its accumulators are complete, so passing this barrier means
+  // every CTA of the cluster is done with its ring and operand tiles (the receive buffer overlays
+  // them); the epilogue warps then observe `done` themselves (already complete: one probe) before
+  // reading the accumulators
   tc_fence_before();
   if (S > 1) {
-    cluster_arrive_relaxed();   // this CTA's MMAs are complete (or it never had any)
+    cluster_arrive_relaxed();
     cluster_wait();
   } else {
     __syncthreads();
   }
   if (warp >= 2) {
+    mbar_wait(done, 0, p.status, DEV_ERR_TIMEOUT_MMA);
     tc_fence_after();
     const int quarter = warp & 3;            // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;
@@ -443,16 +472,28 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
       const int lr = 2 * (pr - q0) + (row & 1);
       float* dst_local = recv + ((size_t)r * rmax + lr) * RST;
       float* dst = S > 1 ? map_peer_w(dst_local, (uint32_t)q) : dst_local;
-      for (int c0 = 0; c0 < NT; c0 += 16) {
-        float vl[16];
+      // 32 columns (hi and lo) per TMEM round trip
+      for (int c0 = 0; c0 < NT; c0 += 32) {
+        float vl[16], v2[16], l2[16];
+        const bool two = c0 + 16 < NT;          // NT is a multiple of 16: warp-uniform
         const uint32_t ta = tmem_d + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(j * 2 * NT + c0);
         tmem_ld16(ta, vals);
         tmem_ld16(ta + (uint32_t)NT, vl);
+        if (two) {
+          tmem_ld16(ta + 16u, v2);
+          tmem_ld16(ta + (uint32_t)NT + 16u, l2);
+        }
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 16; c += 4)
           *reinterpret_cast<float4*>(dst + c0 + c) =
               make_float4(vals[c] + vl[c], vals[c + 1] + vl[c + 1], vals[c + 2] + vl[c + 2], vals[c + 3] + vl[c + 3]);
+        if (two) {
+#pragma unroll
+          for (int c = 0; c < 16; c += 4)
+            *reinterpret_cast<float4*>(dst + c0 + 16 + c) =
+                make_float4(v2[c] + l2[c], v2[c + 1] + l2[c + 1], v2[c + 2] + l2[c + 2], v2[c + 3] + l2[c + 3]);
+        }
       }
     }
   }
@@ -557,7 +598,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
             }
           }
         }
-        sq[col * noct + oc] = hsq;
+        // one owned octet: this unit is its column's only one, so its sum is the CTA's part and
+        // no barrier is needed to collect it
+        if (noct == 1) {
+          if (t < p.Ntok) p.ss_out[(size_t)(mg * S + r) * p.Ntok + t] = hsq;
+        } else {
+          sq[col * noct + oc] = hsq;
+        }
       } else if (EPI == EPI_SWIGLU) {
         if (valid) {
           // rows (2j, 2j+1) = (gate_j, up_j): 8 consecutive intermediate indices = one 16-byte chunk
@@ -633,8 +680,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_stream_kernel(const __gr
         }
       }
     }
-    if (EPI == EPI_RESID) {
-      math_bar();
+    if (EPI == EPI_RESID && noct != 1) {
+      if (noct > 1) math_bar();
       for (int col = mtid; col < NT; col += kMathThreads) {
         const int t = nt * NT + col;
         if (t < p.Ntok) {

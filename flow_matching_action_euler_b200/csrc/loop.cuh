@@ -201,7 +201,9 @@ __global__ void __launch_bounds__(kLoopThreads, 1) loop_kernel(const __grid_cons
     // ------------------------------------------------------------ producer: weight stream
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      int it = 0;
+      int it = 0;                 // tiles issued so far
+      int ps = 0;                 // ring stage of tile `it`
+      uint32_t pph = 0;           // round parity of that stage (tile it uses round it / stages)
       bool ok = true;
       for (int l = p.l0; l < p.l1 && ok; ++l) {
         // the prefix K / V^T rows this CTA's attention units will read in layer l: into L2 now,
@@ -225,16 +227,25 @@ __global__ void __launch_bounds__(kLoopThreads, 1) loop_kernel(const __grid_cons
           if ((int)(task >> 24) == PH_ATTN || !active(l, (int)(task >> 24))) continue;
           const Unit u = unit_of(task);
           const LoopOp& o = p.op[u.op];
-          const uint8_t* base = p.wpack + (size_t)l * p.layer_wbytes + o.woff;
+          const uint8_t* src = p.wpack + (size_t)l * p.layer_wbytes + o.woff +
+                               ((size_t)u.mt0 * o.KBt + u.kt0) * kTileBytes;
+          int li = 0;
           for (int i = 0; i < u.nmt * u.nkt; ++i, ++it) {
-            const int s = it % p.stages;
-            if (it >= p.stages &&
-                !(ok = loop_mbar_wait(&empty[s], ((it / p.stages) - 1) & 1, abort_word, p.status, DEV_ERR_TIMEOUT_TMA)))
+            // stage ps is reused once its previous round (parity pph ^ 1) was consumed
+            if (it >= p.stages && !mbar_try_wait(&empty[ps], pph ^ 1u) &&
+                !(ok = loop_mbar_wait(&empty[ps], pph ^ 1u, abort_word, p.status, DEV_ERR_TIMEOUT_TMA)))
               break;
-            mbar_arrive_expect_tx(&full[s], kTileBytes);
-            bulk_g2s(ring + (size_t)s * kTileBytes,
-                     base + ((size_t)(u.mt0 + i / u.nkt) * o.KBt + u.kt0 + i % u.nkt) * kTileBytes, kTileBytes,
-                     &full[s], pol);
+            mbar_arrive_expect_tx(&full[ps], kTileBytes);
+            bulk_g2s(ring + (size_t)ps * kTileBytes, src, kTileBytes, &full[ps], pol);
+            src += kTileBytes;
+            if (++li == u.nkt) {   // next m-tile of the unit: skip the k-tiles of the other splits
+              li = 0;
+              src += (size_t)(o.KBt - u.nkt) * kTileBytes;
+            }
+            if (++ps == p.stages) {
+              ps = 0;
+              pph ^= 1u;
+            }
           }
         }
       }
@@ -247,9 +258,13 @@ __global__ void __launch_bounds__(kLoopThreads, 1) loop_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 2 * NT);   // hi and lo token rows in one MMA
-      const uint32_t bBase = smem_u32(opb), aBase = smem_u32(ring);
+      // descriptors of ring stage 0 and of the operand's first k-block; 16 bytes = one unit of
+      // the start-address field (shared addresses stay below 256 KB: no carry out of it)
+      const uint64_t a0 = sw128_desc(smem_u32(ring)), b0 = sw128_desc(smem_u32(opb));
       const uint32_t bstride = (uint32_t)NT * 128u;         // bytes of one hi or lo tile
       int it = 0, tcount = 0, opcount = 0, waited = -1;
+      int rs = 0;                                           // ring stage of tile `it`
+      uint32_t rph = 0;                                     // and its phase parity
       bool ok = true;
       for (int l = p.l0; l < p.l1 && ok; ++l) {
         for (int ti = 0; ti < ntask && ok; ++ti) {
@@ -280,19 +295,28 @@ __global__ void __launch_bounds__(kLoopThreads, 1) loop_kernel(const __grid_cons
               !(ok = loop_mbar_wait(&tempty[buf], ((tcount >> 1) - 1) & 1, abort_word, p.status, DEV_ERR_TIMEOUT_MMA)))
             break;
           tc_fence_after();
-          const uint32_t d_base = tmem_d + (uint32_t)(buf * p.acc_cols);
+          // one thread issues every MMA of the CTA: keep the per-tile work to a ring-stage step
+          // (no divisions) and the wait's fast path inline
+          uint32_t d_tmem = tmem_d + (uint32_t)(buf * p.acc_cols);
+          int li = 0;
           for (int i = 0; i < u.nmt * u.nkt; ++i, ++it) {
-            const int s = it % p.stages;
             // the mbarrier orders the bulk-copied tile before the MMA reads it (both async proxy)
-            if (!(ok = loop_mbar_wait(&full[s], (it / p.stages) & 1, abort_word, p.status, DEV_ERR_TIMEOUT_TMA)))
+            if (!mbar_try_wait(&full[rs], rph) &&
+                !(ok = loop_mbar_wait(&full[rs], rph, abort_word, p.status, DEV_ERR_TIMEOUT_TMA)))
               break;
-            const int j = i / u.nkt, li = i % u.nkt;
-            const uint32_t d_tmem = d_base + (uint32_t)(j * 2 * NT);
+            const uint64_t ad = a0 + (uint64_t)((uint32_t)rs * (kTileBytes >> 4));
+            const uint64_t bd = b0 + (uint64_t)((uint32_t)li * 2u * (bstride >> 4));
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(d_tmem, sw128_desc(aBase + s * kTileBytes + kk * 32),
-                       sw128_desc(bBase + (uint32_t)li * 2u * bstride + kk * 32), idesc, (li | kk) != 0);
-            mma_commit(&empty[s]);
+            for (int kk = 0; kk < 4; ++kk) mma_bf16(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (li | kk) != 0);
+            mma_commit(&empty[rs]);
+            if (++rs == p.stages) {
+              rs = 0;
+              rph ^= 1u;
+            }
+            if (++li == u.nkt) {
+              li = 0;
+              d_tmem += (uint32_t)(2 * NT);
+            }
           }
           if (!ok) break;
           mma_commit(&tfull[buf]);

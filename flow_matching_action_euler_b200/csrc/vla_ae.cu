@@ -69,6 +69,8 @@ struct StepTables {
   std::vector<float> dt;    // Euler step k: t_{k+1} - t_k
   // captured graphs, one per (first step, end step, prefix slot, prefix length, engine)
   std::map<std::array<int, 5>, cudaGraphExec_t> graphs;
+  // VLA_AE_ENGINE_AUTO: the engine that ran the whole loop faster, per prefix length
+  std::map<int, bool> auto_loop;
 };
 
 // One prefix buffer set: the layer caches (prefix rows + the self rows the loop writes), the
@@ -93,7 +95,8 @@ struct vla_ae {
   AttnParams attn_proto{};    // attention launch shape: S, span, nrb, Rpad, rpo, smem offsets
   // persistent engine
   bool loop_ok = false;       // planned (bf16, one n-tile, units fit the SMs)
-  bool use_loop = false;      // selected
+  bool use_loop = false;      // selected (the engine the next capture uses)
+  int engine_mode = VLA_AE_ENGINE_PER_OP;   // as set by vla_ae_set_engine
   int loop_cs = 16;           // attention sub-chunk of the persistent kernel
   LoopParams loop_proto{};    // plan: op shapes, smem layout, task lists, scratch
   size_t ctr_step = 0;        // counters per launch (layers x ctr_layer + abort word)
@@ -1476,14 +1479,69 @@ int vla_ae_set_prefix_next(vla_ae_t H, const void* k, const void* v, int n_prefi
   return VLA_AE_OK;
 }
 
+// VLA_AE_ENGINE_AUTO: on the first whole loop of T at the current prefix length, capture the loop
+// with both engines and time a few replays of each on `st` (queued after the caller's noise copy,
+// so they compute the very loop the caller asked for: every buffer a replay writes is rewritten by
+// the launch that follows); the faster engine is kept for T and that prefix length.
+static int auto_engine(vla_ae_t H, StepTables* T, cudaStream_t st) {
+  const int key = H->slot[H->front].n_prefix;
+  auto it = T->auto_loop.find(key);
+  if (it != T->auto_loop.end()) {
+    H->use_loop = it->second;
+    return VLA_AE_OK;
+  }
+  if (!H->loop_ok) {
+    H->use_loop = false;
+    T->auto_loop.emplace(key, false);
+    return VLA_AE_OK;
+  }
+  cudaEvent_t ev[2] = {nullptr, nullptr};
+  if (cudaEventCreate(&ev[0]) != cudaSuccess || cudaEventCreate(&ev[1]) != cudaSuccess) {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);
+    cudaGetLastError();
+    return VLA_AE_ECUDA;
+  }
+  float best = 0.f;
+  bool pick = false;
+  int rc = VLA_AE_OK;
+  for (int lp = 0; lp < 2 && rc == VLA_AE_OK; ++lp) {
+    H->use_loop = lp == 1;
+    cudaGraphExec_t exec = nullptr;
+    if ((rc = ensure_graph(H, T, 0, T->steps, H->front, &exec))) break;
+    float ms = 0.f;
+    if (cudaGraphLaunch(exec, st) != cudaSuccess || cudaEventRecord(ev[0], st) != cudaSuccess) rc = VLA_AE_ECUDA;
+    for (int r = 0; r < 3 && rc == VLA_AE_OK; ++r)
+      if (cudaGraphLaunch(exec, st) != cudaSuccess) rc = VLA_AE_ECUDA;
+    if (rc == VLA_AE_OK && (cudaEventRecord(ev[1], st) != cudaSuccess || cudaEventSynchronize(ev[1]) != cudaSuccess ||
+                            cudaEventElapsedTime(&ms, ev[0], ev[1]) != cudaSuccess))
+      rc = VLA_AE_ECUDA;
+    if (rc == VLA_AE_OK && (lp == 0 || ms < best)) {
+      best = ms;
+      pick = lp == 1;
+    }
+  }
+  cudaEventDestroy(ev[0]);
+  cudaEventDestroy(ev[1]);
+  if (rc) {
+    cudaGetLastError();
+    H->use_loop = false;
+    return rc;
+  }
+  H->use_loop = pick;
+  T->auto_loop.emplace(key, pick);
+  return VLA_AE_OK;
+}
+
 static int denoise_tables(vla_ae_t H, StepTables* T, const void* noise, float* out, void* stream, bool host) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaGraphExec_t exec = nullptr;
   int rc;
-  if ((rc = ensure_graph(H, T, 0, T->steps, H->front, &exec))) return rc;
   const vla_ae_dims& d = H->d;
   const size_t nx = (size_t)d.batch * d.n_action_tokens * d.action_dim;
   CK(cudaMemcpyAsync(H->noise_stage, noise, nx * 2, host ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, st));
+  if (H->engine_mode == VLA_AE_ENGINE_AUTO && (rc = auto_engine(H, T, st))) return rc;
+  if ((rc = ensure_graph(H, T, 0, T->steps, H->front, &exec))) return rc;
   CK(cudaGraphLaunch(exec, st));
   CK(cudaMemcpyAsync(out, H->out_stage, nx * 4, host ? cudaMemcpyDeviceToHost : cudaMemcpyDeviceToDevice, st));
   return VLA_AE_OK;
@@ -1514,6 +1572,10 @@ int vla_ae_denoise_stale(vla_ae_t H, const void* noise, int steps, int n_stale, 
   int rc = get_tables(H, steps, &T);
   if (rc) return rc;
   const int back = 1 - H->front;
+  if (H->engine_mode == VLA_AE_ENGINE_AUTO) {   // the choice made for whole loops, if any
+    auto it = T->auto_loop.find(H->slot[H->front].n_prefix);
+    H->use_loop = it != T->auto_loop.end() && it->second;
+  }
   cudaGraphExec_t ga = nullptr, gb = nullptr;
   if (n_stale > 0 && (rc = ensure_graph(H, T, 0, n_stale, H->front, &ga))) return rc;
   if (n_stale < steps && (rc = ensure_graph(H, T, n_stale, steps, back, &gb))) return rc;
@@ -1610,9 +1672,13 @@ int vla_ae_bench_op(vla_ae_t H, int op, int count, int steps, void* stream) {
 }
 
 int vla_ae_set_engine(vla_ae_t H, int engine) {
-  if (!H || (engine != VLA_AE_ENGINE_PER_OP && engine != VLA_AE_ENGINE_PERSISTENT)) return VLA_AE_EINVAL;
+  if (!H || (engine != VLA_AE_ENGINE_PER_OP && engine != VLA_AE_ENGINE_PERSISTENT && engine != VLA_AE_ENGINE_AUTO))
+    return VLA_AE_EINVAL;
   if (engine == VLA_AE_ENGINE_PERSISTENT && !H->loop_ok) return VLA_AE_EUNSUPPORTED;
-  H->use_loop = engine == VLA_AE_ENGINE_PERSISTENT;   // graphs re-capture on their next use
+  H->engine_mode = engine;
+  // graphs of the other engine re-capture on their next use; AUTO keeps the current engine until
+  // its first whole loop decides
+  if (engine != VLA_AE_ENGINE_AUTO) H->use_loop = engine == VLA_AE_ENGINE_PERSISTENT;
   return VLA_AE_OK;
 }
 

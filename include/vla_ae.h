@@ -246,11 +246,18 @@ int vla_ae_bench_op(vla_ae_t h, int op, int count, int steps, void *stream);
  *     layers; weights stream continuously and phases hand over through device-scope counters.
  *     Available for bf16 weights with at most 128 token rows (batch x self tokens), a hidden
  *     size that is a multiple of 4, and work units that fit the SMs.
+ *   VLA_AE_ENGINE_AUTO (2): the first vla_ae_denoise / _host / _sched call of a step count (or
+ *     time grid) and prefix length captures the loop with both engines, times three replays of
+ *     each on the caller's stream (a one-off cost of a few loops, synchronising the host once) and
+ *     keeps the faster; later calls replay it.  vla_ae_denoise_stale follows the choice made for
+ *     whole loops (per-op until one was made).  Without the persistent engine, AUTO is per-op.
  * create selects VLA_AE_ENGINE_PER_OP.
  * Select the engine for later denoise / debug calls (a graph captured for the other engine is
- * re-captured).  Errors: EINVAL, EUNSUPPORTED (persistent engine not available here). */
+ * re-captured); VLA_AE_Q_ENGINE reports the engine in use (AUTO: the one it picked).
+ * Errors: EINVAL, EUNSUPPORTED (persistent engine not available here). */
 #define VLA_AE_ENGINE_PER_OP 0
 #define VLA_AE_ENGINE_PERSISTENT 1
+#define VLA_AE_ENGINE_AUTO 2
 int vla_ae_set_engine(vla_ae_t h, int engine);
 
 /* ------------------------------------------------------------------ test hooks

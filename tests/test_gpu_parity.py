@@ -206,6 +206,30 @@ def test_engine_selection():
     assert e.value.code == fm.EINVAL
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_engine_auto(name):
+    """AUTO times both engines on the first whole loop, keeps the faster one, and the result is
+    that engine's: bit-identical to running it by hand, and within tolerance of the oracle."""
+    import flow_matching_action_euler_b200 as fm
+    c = case(name)
+    ref = c.oracle_denoise()
+    with engine(c, fm.ENGINE_AUTO):
+        auto = c.denoise()
+        picked = c.ae.engine
+        assert picked in (fm.ENGINE_PER_OP, fm.ENGINE_PERSISTENT)
+        again = c.denoise()                                        # replays the kept graph
+        assert c.ae.engine == picked
+        assert np.array_equal(auto, again)
+    with engine(c, picked):
+        by_hand = c.denoise()
+    assert np.array_equal(auto, by_hand)
+    assert rel_err(auto, ref) <= FINAL_TOL
+    c8 = case("tiny", wtype="fp8_e4m3")                            # no persistent engine: per-op
+    with engine(c8, fm.ENGINE_AUTO):
+        c8.denoise()
+        assert c8.ae.engine == fm.ENGINE_PER_OP
+
+
 def _denoise_sched(c, grid):
     d = c.d
     from tests.gpu_util import bits_to_cuda
