@@ -36,7 +36,8 @@ METRIC = "action-expert denoise-loop ms and achieved HBM GB/s at batch 1 (1x B20
 FALLBACK_HBM_GBS = 6650.0
 OP_NAMES = ("qkv_rope", "attention", "o_proj_resid", "gate_up_swiglu", "down_resid")
 DOMINANT_OP = 3
-KERNEL_SOURCES = ("ptx.cuh", "gemm.cuh")
+# the dominant kernel's source and the host code that plans its launch shape (split, ring depth)
+KERNEL_SOURCES = ("ptx.cuh", "gemm.cuh", "vla_ae.cu")
 
 
 def parse_args():

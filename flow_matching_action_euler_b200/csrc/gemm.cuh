@@ -10,8 +10,9 @@
 //    128 e4m3) already laid out in the 128-byte swizzle the MMA reads, stored [m-tile][k-block]
 //    so every CTA's share is one contiguous range per m-tile, fetched with 1-D bulk copies;
 //  * the producer warp issues those copies before `griddepcontrol.wait`, i.e. while the previous
-//    kernel of the loop is still running (programmatic dependent launch); 192 threads and
-//    ~110 KB of shared memory let two CTAs share an SM so the overlap really happens;
+//    kernel of the loop is still running (programmatic dependent launch), on the SMs that kernel
+//    leaves free; the ring is as deep as the CTA's share of tiles (up to 8 stages, most of the
+//    SM's shared memory), which measured faster than two shallower CTAs per SM;
 //  * the activation operand is a pair of bf16 tiles (hi, lo = x - hi) written by the producing
 //    kernel in the swizzled layout and fetched with one bulk copy; the two tiles are adjacent, so
 //    one MMA with N = 2 NT multiplies both (on B200 an M=128 MMA costs the same ~58 cycles for
