@@ -305,7 +305,11 @@ bool cluster_fits(GemmKernel kern, const OpPlan& p, int Nt, bool one_wave) {
 }
 
 // Choose m-tiles per CTA and the split so that one wave of CTAs covers the GPU with the
-// fewest weight tiles per CTA, inside the shared-memory budget.
+// fewest weight tiles per CTA, inside the shared-memory budget.  When no single-wave plan exists
+// (many token tiles: large batches, the prefix producer), minimise an estimate of the launch's
+// time instead: waves x per-CTA time, the latter in units of one resident tile's MMAs (~0.26 us):
+// a fixed ~6 us per CTA (launch, operand, split-K exchange, epilogue), the tiles (slower when a
+// shallow ring leaves L2 latency exposed) and the split-K push of the CTA's accumulators.
 // Split / m-group / ring plan of one GEMM over Nt token tiles of NT rows with weight format wq.
 int plan_gemm_shape(vla_ae* H, OpPlan& out, OpId id, int O, int K, int NT, int Nt, int wq) {
   const bool fp8 = wq != 0;
@@ -352,8 +356,16 @@ int plan_gemm_shape(vla_ae* H, OpPlan& out, OpId id, int O, int K, int NT, int N
         }
         if (p.smem > kMaxDynSmem) continue;
         const int over = p.smem > (fp8 ? kMaxDynSmem : budget) ? 1 : 0;
-        // lexicographic: inside budget, fewest tiles per CTA, smallest split, fewest m-tiles per CTA
-        const long key = (long)over * 1000000 + (long)tiles * 1000 + S * 10 + mpc;
+        // one wave: lexicographic (inside budget, fewest tiles per CTA, smallest split, fewest
+        // m-tiles per CTA); several waves: estimated time first
+        long cost = 0;
+        if (pass == 1) {
+          const int per_sm = (p.smem <= kMaxDynSmem / 2 - 1024 && mpc * 2 * NT <= 256) ? 2 : 1;
+          const long waves = ceil_div(ctas, H->num_sms * per_sm);
+          const double cta = 24.0 + tiles * std::max(1.0, 4.0 / p.stages) + (S > 1 ? mpc * NT / 48.0 : 0.0);
+          cost = (long)(waves * cta * 100.0);
+        }
+        const long key = (long)over * 10000000000000L + cost * 1000000L + (long)tiles * 1000 + S * 10 + mpc;
         if (found && key >= best_key) continue;
         if (!cluster_fits(kern, p, Nt, pass == 0)) continue;
         best = p;

@@ -85,6 +85,22 @@ def test_full_size_fp8(wtype, steps):
         c.close()
 
 
+def test_starvla_int4_several_k_tiles():
+    """StarVLA-shaped loop (1 Euler step) on INT4 weights.  Its down-projection (1536 rows,
+    K = 4096: 16 packed k-tiles) cannot give every K split a single packed tile inside one wave of
+    CTAs, so each CTA walks several k-tiles of widened weights: the operand k-blocks of each must
+    follow the tile's width (4 k-blocks per int4 tile)."""
+    import flow_matching_action_euler_b200 as fm
+    c = Case(config("starvla", wtype="int4_g128", steps=1))
+    try:
+        s_down = (c.ae.query(fm.Q_SPLITS) >> 24) & 0xFF
+        assert 16 > s_down                            # more packed k-tiles than splits
+        got = c.denoise()
+        assert rel_err(got, c.oracle_denoise()) <= 2e-2
+    finally:
+        c.close()
+
+
 def test_pi05_one_step_variant():
     """The one-step action generation of the APXInf article on the pi0.5 shape: grid {1, 0}."""
     import torch
