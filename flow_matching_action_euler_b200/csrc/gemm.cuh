@@ -15,9 +15,10 @@
 //    SM's shared memory), which measured faster than two shallower CTAs per SM;
 //  * the activation operand is a pair of bf16 tiles (hi, lo = x - hi) written by the producing
 //    kernel in the swizzled layout and fetched with one bulk copy; the two tiles are adjacent, so
-//    one MMA with N = 2 NT multiplies both (on B200 an M=128 MMA costs the same ~58 cycles for
-//    any N <= 64) and the epilogue adds the two column halves: the product is fp32-accurate in
-//    the activations while the weights stay exact bf16;
+//    one MMA with N = 2 NT multiplies both (measured on B200: a 16 KB tile's four M=128 K=16 MMAs
+//    take ~350 cycles at N = 64 and ~500 at N = 256, so the lo rows cost little) and the epilogue
+//    adds the two column halves: the product is fp32-accurate in the activations while the
+//    weights stay exact bf16;
 //  * RMSNorm + adaLN modulate ("AI Infra如何优化VLA" section 算子开发) are applied by linearity:
 //    W (rms(h) (1 + scale) + shift) = rstd * W (h (1 + scale)) + W shift, so producers write
 //    h (1 + scale), this kernel scales by rstd (from partial sums of squares) in the epilogue and

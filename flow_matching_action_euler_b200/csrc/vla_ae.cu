@@ -333,7 +333,8 @@ int plan_gemm_shape(vla_ae* H, OpPlan& out, OpId id, int O, int K, int NT, int N
   long best_key = 0;
   for (int pass = 0; pass < 2 && !found; ++pass) {      // pass 1 allows more than one wave
     for (int mpc : {1, 2, 4}) {
-      // TMEM: half of it (room for a second CTA per SM), or all of it in the fallback pass
+      // TMEM: half of it (room for a dependent kernel's CTA beside this one), or all of it in
+      // the several-wave pass
       if (mpc > base.Mt || mpc * 2 * NT > (pass == 0 ? 256 : 512)) continue;
       const int mg = ceil_div(base.Mt, mpc);
       for (int S = 1; S <= std::min(16, base.KBt); ++S) {
