@@ -338,15 +338,20 @@ def run_native(args):
         torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    # one event between consecutive loops: the total over all K gives the line's time, the
+    # per-loop spans its spread (median, p10, p90)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record(stream)
+    for i in range(args.steps):
         ae.denoise(noise, N, out, stream)
-    e1.record(stream)
+        evs[i + 1].record(stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, "cuda")
+    ms = max_over_ranks(evs[0].elapsed_time(evs[-1]) / args.steps, world, "cuda")
+    per_loop = sorted(evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps))
+    loop_dist = {q: round(per_loop[min(len(per_loop) - 1, int(f * len(per_loop)))], 5)
+                 for q, f in (("p10", 0.1), ("p50", 0.5), ("p90", 0.9))}
     if ae.status() != 0:
         raise RuntimeError("device-side timeout during the timed region")
 
@@ -362,6 +367,7 @@ def run_native(args):
                   "int4_g128": "int4 weights (groups of 128) x bf16 activations"}[d.wtype],
         "data": "synthetic", "config": workload_config(d, args), "engine": engine,
         "ms_per_loop": round(ms, 5),
+        "ms_per_loop_dist": dict(loop_dist, rank=0),
         "actions_per_s": round(world * d.batch * d.n_action_tokens * 1000.0 / ms, 1),
         "chunks_per_s": round(world * d.batch * 1000.0 / ms, 2),
         "hbm_frac_of_8tbs": round(value / world / 8000.0, 4),
