@@ -39,7 +39,10 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
 ``prefix_kv``          composed of the pinned rms_norm / linear / rope_half;
                        invariant to scaling h; position 0 is the plain projection
 ``dit_layer``          zero gates give the identity, joint prefix permutation
-                       invariance
+                       invariance, self-token permutation equivariance, branch
+                       isolation under each adaLN gate, and the closed form of
+                       uniform attention (W_q = 0: each head outputs the mean of
+                       its kv group's prefix + self value rows)
 ``velocity``/``denoise``  parity unpinned beyond the parts above: batch
                        independence (bitwise), determinism
 =====================  =========================================================

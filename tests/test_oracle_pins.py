@@ -515,6 +515,36 @@ def test_layer_branch_isolation_under_zero_gates():
     assert np.max(np.abs(oracle.dit_layer(h, lw, mod, kp, vp, pos, d) - base)) > 1e-6
 
 
+def test_layer_uniform_attention_closed_form():
+    """W_q = 0 makes every score 0, so each query head's softmax is uniform over the P + Ts keys
+    and its output is the plain mean of its kv group's value rows: the prefix V rows and the
+    self rows v = W_v u (not rotated), u = RMSNorm(h) (1 + scale_a) + shift_a.  With the MLP gate
+    closed the layer is then h + gate_a * W_o o, written out here with einsum on that closed
+    form (no softmax), which pins the adaLN chunk order of the attention branch, the GQA
+    head-to-group map and the prefix + self key set."""
+    d = MICRO
+    W, lw, mod, kp, vp, h, pos = _layer_inputs(d, seed=5)
+    H, hd, nq, nkv = d.hidden, d.head_dim, d.n_q_heads, d.n_kv_heads
+    lw = dict(lw)
+    lw["wq"] = np.zeros_like(lw["wq"])
+    mod = mod.copy()
+    mod[5 * H:6 * H] = 0.0                                    # gate_m: MLP branch off
+    shift_a, scale_a, gate_a = mod[0:H], mod[H:2 * H], mod[2 * H:3 * H]
+    ms = np.mean(h * h, axis=1, keepdims=True)
+    u = h / np.sqrt(ms + d.rms_eps) * (1.0 + scale_a) + shift_a
+    v_self = np.einsum("ok,tk->to", lw["wv"], u).reshape(d.ts, nkv, hd)
+    v_all = np.concatenate([vp, v_self], axis=0)              # [P + Ts, nkv, hd]
+    mean_v = v_all.mean(axis=0)                               # [nkv, hd]
+    o = np.stack([mean_v[qh // (nq // nkv)] for qh in range(nq)]).reshape(-1)   # [nq * hd]
+    want = h + gate_a * np.einsum("ok,k->o", lw["wo"], o)[None, :]
+    got = oracle.dit_layer(h, lw, mod, kp, vp, pos, d)
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-12)
+    # the group map matters: a wrong head-to-group assignment changes the result
+    o_bad = np.stack([mean_v[qh % nkv] for qh in range(nq)]).reshape(-1)
+    bad = h + gate_a * np.einsum("ok,k->o", lw["wo"], o_bad)[None, :]
+    assert np.max(np.abs(bad - got)) > 1e-6
+
+
 # ----------------------------------------------------------------- INT8 weights (row-wise)
 
 def test_int8_max_entry_maps_to_127_and_codes_are_bounded():
