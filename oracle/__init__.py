@@ -43,8 +43,12 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
                        isolation under each adaLN gate, and the closed form of
                        uniform attention (W_q = 0: each head outputs the mean of
                        its kv group's prefix + self value rows)
-``velocity``/``denoise``  parity unpinned beyond the parts above: batch
-                       independence (bitwise), determinism
+``velocity``           closed form with every adaLN gate and the final
+                       modulation zero (W_out RMSNorm(W_in x + b_in) + b_out on the
+                       action rows, the state row dropped); one step of
+                       ``denoise`` is one Euler update of it
+``denoise``            batch independence (bitwise), determinism; the loop is
+                       ``euler_integrate``'s, pinned above
 =====================  =========================================================
 """
 

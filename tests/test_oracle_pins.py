@@ -447,6 +447,39 @@ def test_batch_independence_bitwise_and_determinism():
     assert np.array_equal(again, full)
 
 
+def test_velocity_with_closed_gates_closed_form():
+    """All adaLN gates and the final modulation zero: every DiT layer is the identity, so the
+    velocity of action row j is W_out RMSNorm(W_in x_j + b_in) + b_out, the state row (first) being
+    dropped.  Written here with einsum on that closed form; pins the in/out projection
+    orientation, the per-row final norm, the biases and which row is dropped."""
+    d = MICRO
+    w = generate_weights(d, 0)
+    x = generate_inputs(d, 0)
+    H = d.hidden
+    w = dict(w)
+    w["layers"] = [dict(lw) for lw in w["layers"]]
+    for lw in w["layers"]:
+        for key in ("w_ada", "b_ada"):
+            a = lw[key].copy()
+            a[2 * H:3 * H] = 0                                   # gate_a (bf16 +0)
+            a[5 * H:6 * H] = 0                                   # gate_m
+            lw[key] = a
+    w["w_fada"] = np.zeros_like(w["w_fada"])
+    w["b_fada"] = np.zeros_like(w["b_fada"])
+    W = oracle.OracleWeights(w, d)
+    xs = oracle.bf16_to_f64(x["noise"][0])
+    st = oracle.bf16_to_f64(x["state"][0])
+    kp, vp = oracle.bf16_to_f64(x["k"][0]), oracle.bf16_to_f64(x["v"][0])
+    got = oracle.velocity(xs, 0.4, st, W, kp, vp, d)
+    top = {k: oracle.bf16_to_f64(w[k]) for k in ("w_in", "b_in", "w_out", "b_out")}
+    h = np.einsum("ha,ta->th", top["w_in"], xs) + top["b_in"]
+    u = h / np.sqrt(np.mean(h * h, axis=1, keepdims=True) + d.rms_eps)
+    want = np.einsum("ah,th->ta", top["w_out"], u) + top["b_out"]
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+    # the prefix and the time no longer matter
+    np.testing.assert_allclose(oracle.velocity(xs, 0.9, st, W, kp + 1.0, vp * 2.0, d), got, rtol=1e-12, atol=1e-13)
+
+
 def test_single_step_is_one_euler_update():
     d = MICRO
     w = generate_weights(d, 0)
