@@ -22,6 +22,8 @@ Functions and what pins them (tests under ``tests/test_oracle_*.py``):
                        n_stale = 0 / N reduce to one field
 ``timestep_embedding`` t = 0 gives [1..1, 0..0]; first frequency is 1000 t;
                        last frequency matches the base-10000 geometric series
+``adaln_table``        closed form at t = 0 (SiLU(1) x row sums of the cos half of
+                       W_ada, plus b_ada)
 ``rms_norm``           unit RMS at eps = 0, scale invariance, torch's rms_norm
 ``modulate``           shift = scale = 0 is the identity
 ``rope_half``          per-pair norm, position 0 identity, relative-position

@@ -400,6 +400,20 @@ def _layer_inputs(d, seed=0):
     return W, lw, mod, kp, vp, h, pos
 
 
+def test_adaln_table_at_t0_closed_form():
+    """At t = 0 the embedding is [cos 0 .. | sin 0 ..] = [1 .. 1 | 0 .. 0], so the modulation is
+    SiLU(1) times the row sums of W_ada's first half of columns, plus b_ada (SiLU(1) = 1 / (1 +
+    1/e)).  Pins the [cos | sin] order, the SiLU before the projection, W_ada's orientation and
+    the bias."""
+    rng = np.random.default_rng(21)
+    dt_dim, rows = 16, 12
+    w = rng.standard_normal((rows, dt_dim))
+    b = rng.standard_normal(rows)
+    silu1 = 1.0 / (1.0 + math.exp(-1.0))
+    want = silu1 * w[:, :dt_dim // 2].sum(axis=1) + b
+    np.testing.assert_allclose(oracle.adaln_table(w, b, 0.0, dt_dim), want, rtol=1e-14, atol=1e-14)
+
+
 def test_layer_zero_gates_is_identity():
     d = MICRO
     W, lw, mod, kp, vp, h, pos = _layer_inputs(d)
