@@ -37,7 +37,7 @@ extern "C" {
 #define VLA_AE_ECUDA (-3)        /* a CUDA runtime call failed (no device, launch error, ...) */
 #define VLA_AE_ENOPREFIX (-4)    /* vla_ae_denoise before any vla_ae_set_prefix */
 #define VLA_AE_ETIMEOUT (-5)     /* a bounded device-side wait ran out (see vla_ae_status) */
-#define VLA_AE_EUNSUPPORTED (-6) /* valid dims this build does not implement (e.g. head_dim) */
+#define VLA_AE_EUNSUPPORTED (-6) /* valid dims the library does not implement (e.g. head_dim) */
 
 /* ------------------------------------------------------------------ configuration */
 /* Weight formats of the per-layer linears.  FP8_E4M3: the FP8 weights of the APXInf article
